@@ -1,0 +1,535 @@
+#!/usr/bin/env python
+"""Benchmark of the TQ3 KV-cache codec (and, on request, the RPBH weight path) on B200.
+
+Default workload: a bf16 KV cache, K and V each [batch 8, kv_heads 8, seq 4096, head_dim 128]
+(524,288 vectors of 128), N(0,1) plus 4 outlier channels x20 and a per-token N(0, 2^2) offset,
+seed 1. One step encodes K and V to TQ3 records and decodes both back to bf16:
+encode(K), encode(V), decode(K), decode(V). Inputs are resident in HBM; every kernel reads data
+last touched at least one 160 MB kernel earlier, so no input is served from the 126 MB L2.
+
+Prints ONE JSON line (rank 0). `value` = vectors encoded and decoded per second over all ranks
+(each rank runs its own full cache: weak scaling, no data-path collective). `e2e` is the same
+metric with K and V copied in from pinned host memory and the decoded caches plus the TQ3 records
+copied back every step. `cpu_baseline` times the single-threaded C oracle on a bounded sample of
+the same workload on this host. `--impl reference` times that oracle as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from weight_quantization_b200 import inputs  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+HBM_FALLBACK_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------------------------
+# environment helpers
+# ---------------------------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return HBM_FALLBACK_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.lines:
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def traffic_bytes(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    src = {"tq3_encode": "tq3.cu", "tq3_decode": "tq3.cu", "rpbh_quantize": "rpbh.cu", "rpbh_rotate": "rpbh.cu",
+           "rpbh_dequantize": "rpbh.cu"}.get(kernel)
+    if src is None:
+        return None
+    with open(os.path.join(ROOT, "weight_quantization_b200", "csrc", src), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(p) as f:
+        for line in f:
+            parts = line.split()
+            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == sha:
+                return float(parts[3])
+    return None
+
+
+# ---------------------------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------------------------
+class KVWorkload:
+    """TQ3 encode + decode of a bf16 KV cache (K and V)."""
+
+    name = "tq3-kv-cache-bf16-8x8x4096x128"
+    unit = "vectors/s"
+    metric = "TQ3 encode+decode vectors/s (K and V caches, bf16)"
+
+    def __init__(self, dev, seed=1):
+        from weight_quantization_b200 import ops
+        self.ops = ops
+        k, v = inputs.kv_cache(seed=seed)
+        self.host = [torch.from_numpy(a.reshape(-1, 128).view(np.int16)).view(torch.bfloat16) for a in (k, v)]
+        self.n_half = self.host[0].shape[0]
+        self.units = 2 * self.n_half
+        self.mask = ops.sign_mask_words(inputs.tq3_sign_bits())
+        self.x = [h.to(dev) for h in self.host]
+        self.packed = [torch.empty(self.n_half, 48, dtype=torch.uint8, device=dev) for _ in range(2)]
+        self.norms = [torch.empty(self.n_half, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.scales = [torch.empty(self.n_half, dtype=torch.float32, device=dev) for _ in range(2)]
+        self.out = [torch.empty(self.n_half, 128, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.kernels = ["tq3_encode", "tq3_decode"]
+        self.bytes_per_launch = {"tq3_encode": 312 * self.n_half, "tq3_decode": 312 * self.n_half}
+
+    def step(self, ev=None):
+        o = self.ops
+        for i in range(2):
+            self._mark(ev, "tq3_encode", 0)
+            o.tq3_encode(self.x[i], self.mask, self.packed[i].view(-1, 1, 48), self.norms[i].view(-1, 1),
+                         self.scales[i].view(-1, 1))
+            self._mark(ev, "tq3_encode", 1)
+        for i in range(2):
+            self._mark(ev, "tq3_decode", 0)
+            o.tq3_decode(self.packed[i], self.norms[i], self.scales[i], self.mask, out=self.out[i])
+            self._mark(ev, "tq3_decode", 1)
+        return 4
+
+    @staticmethod
+    def _mark(ev, k, which):
+        if ev is not None:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record()
+            ev.setdefault(k, []).append(e)
+
+    # end to end: pinned host K, V in; decoded K, V and the TQ3 records out
+    def e2e_setup(self):
+        self.pin_in = [h.pin_memory() for h in self.host]
+        self.pin_out = [torch.empty_like(h).pin_memory() for h in self.host]
+        self.pin_packed = [torch.empty(self.n_half, 48, dtype=torch.uint8).pin_memory() for _ in range(2)]
+        self.pin_ns = [torch.empty(2, self.n_half, dtype=torch.float32).pin_memory() for _ in range(2)]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.pin_in)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.pin_out + self.pin_packed + self.pin_ns)
+
+    def e2e_step(self):
+        for i in range(2):
+            self.x[i].copy_(self.pin_in[i], non_blocking=True)
+        self.step()
+        for i in range(2):
+            self.pin_out[i].copy_(self.out[i], non_blocking=True)
+            self.pin_packed[i].copy_(self.packed[i], non_blocking=True)
+            self.pin_ns[i][0].copy_(self.norms[i], non_blocking=True)
+            self.pin_ns[i][1].copy_(self.scales[i], non_blocking=True)
+
+    # the oracle on a bounded sample of the same cache
+    def oracle_rate(self, budget_s=10.0):
+        import oracle
+        oracle.lib()
+        bits = inputs.tq3_sign_bits()
+        src = self.host[0].view(torch.int16).numpy().view(np.uint16)
+        done, t0, chunk = 0, time.perf_counter(), 2048
+        while time.perf_counter() - t0 < budget_s and done + chunk <= src.shape[0]:
+            x = src[done:done + chunk]
+            p, n, s = oracle.tq3_encode(x, bits, is_bf16=True)
+            oracle.tq3_decode(p, n, s, bits, out_bf16=True)
+            done += chunk
+        dt = time.perf_counter() - t0
+        return done / dt, f"first {done} vectors of the K cache, encode + decode to bf16, {dt:.1f} s"
+
+
+class LongContextWorkload(KVWorkload):
+    """Decode-only: 1,048,576 TQ3 records to bf16 [1, 8, 131072, 128]."""
+
+    name = "tq3-decode-long-context-1x8x131072x128"
+    metric = "TQ3 decode vectors/s (1M records to bf16)"
+
+    def __init__(self, dev, seed=2):
+        from weight_quantization_b200 import ops
+        self.ops = ops
+        p, n, s = inputs.long_context_records(seed=seed)
+        self.mask = ops.sign_mask_words(inputs.tq3_sign_bits())
+        self.host_rec = (torch.from_numpy(p), torch.from_numpy(n), torch.from_numpy(s))
+        self.rec = [t.to(dev) for t in self.host_rec]
+        self.n_half = p.shape[0]
+        self.units = self.n_half
+        self.out = torch.empty(self.n_half, 128, dtype=torch.bfloat16, device=dev)
+        self.kernels = ["tq3_decode"]
+        self.bytes_per_launch = {"tq3_decode": 312 * self.n_half}
+
+    def step(self, ev=None):
+        self._mark(ev, "tq3_decode", 0)
+        self.ops.tq3_decode(self.rec[0], self.rec[1], self.rec[2], self.mask, out=self.out)
+        self._mark(ev, "tq3_decode", 1)
+        return 1
+
+    def e2e_setup(self):
+        self.pin_rec = [t.pin_memory() for t in self.host_rec]
+        self.pin_out = torch.empty(self.n_half, 128, dtype=torch.bfloat16).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in self.pin_rec)
+        self.d2h = self.pin_out.numel() * 2
+
+    def e2e_step(self):
+        for d, h in zip(self.rec, self.pin_rec):
+            d.copy_(h, non_blocking=True)
+        self.step()
+        self.pin_out.copy_(self.out, non_blocking=True)
+
+    def oracle_rate(self, budget_s=10.0):
+        import oracle
+        oracle.lib()
+        bits = inputs.tq3_sign_bits()
+        p, n, s = (t.numpy() for t in self.host_rec)
+        done, t0, chunk = 0, time.perf_counter(), 4096
+        while time.perf_counter() - t0 < budget_s and done + chunk <= p.shape[0]:
+            oracle.tq3_decode(p[done:done + chunk], n[done:done + chunk], s[done:done + chunk], bits, out_bf16=True)
+            done += chunk
+        dt = time.perf_counter() - t0
+        return done / dt, f"first {done} records decoded to bf16, {dt:.1f} s"
+
+
+class RPBHWorkload:
+    """RPBH on an LLM MLP weight W[4096, 11008] bf16 (3 bits) and activations x[2048, 11008]:
+    quantize W, dequantize W' (rotated, bf16) and rotate x."""
+
+    metric = "RPBH weight elements/s (quantize + rotated dequantize + activation rotation)"
+    unit = "elements/s"
+
+    def __init__(self, dev, rows=4096, d=11008, xrows=2048, bits=3, seed=3, name=None):
+        from weight_quantization_b200 import ops
+        self.ops = ops
+        self.name = name or f"rpbh-w{rows}x{d}-x{xrows}-b{bits}"
+        w = inputs.llm_weight(rows, d, seed=seed) if d == 11008 else inputs.dit_weight(rows, d, seed=seed)
+        x = inputs.activations(xrows, d, seed=seed)
+        perm, signs = inputs.rpbh_params(d)
+        self.rows, self.d, self.xrows, self.bits = rows, d, xrows, bits
+        bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        self.host = [bf(w), bf(x)]
+        self.w, self.x = (t.to(dev) for t in self.host)
+        self.perm = torch.from_numpy(perm).to(dev)
+        self.signs = torch.from_numpy(signs).to(dev)
+        self.cb = ops.rpbh_codebook(bits, d)
+        self.packed = torch.empty(ops.rpbh_packed_bytes(rows, d, bits), dtype=torch.uint8, device=dev)
+        self.norms = torch.empty(rows, dtype=torch.bfloat16, device=dev)
+        self.wq = torch.empty(rows, d, dtype=torch.bfloat16, device=dev)
+        self.xr = torch.empty(xrows, d, dtype=torch.bfloat16, device=dev)
+        self.units = rows * d
+        self.kernels = ["rpbh_quantize", "rpbh_dequantize", "rpbh_rotate"]
+        n = rows * d
+        self.bytes_per_launch = {"rpbh_quantize": 2 * n + n * bits // 8 + 2 * rows,
+                                 "rpbh_dequantize": 2 * n + n * bits // 8 + 2 * rows,
+                                 "rpbh_rotate": 4 * xrows * d}
+
+    _mark = staticmethod(KVWorkload._mark)
+
+    def step(self, ev=None):
+        o = self.ops
+        self._mark(ev, "rpbh_quantize", 0)
+        o.rpbh_quantize_weight(self.w, self.perm, self.signs, self.bits, self.cb, self.packed, self.norms)
+        self._mark(ev, "rpbh_quantize", 1)
+        self._mark(ev, "rpbh_rotate", 0)
+        o.rpbh_rotate_activations(self.x, self.perm, self.signs, out=self.xr)
+        self._mark(ev, "rpbh_rotate", 1)
+        self._mark(ev, "rpbh_dequantize", 0)
+        o.rpbh_dequantize_weight(self.packed, self.norms, self.rows, self.d, self.bits, self.cb,
+                                 out_dtype=torch.bfloat16, out=self.wq)
+        self._mark(ev, "rpbh_dequantize", 1)
+        return 3
+
+    def e2e_setup(self):
+        self.pin_in = [h.pin_memory() for h in self.host]
+        self.pin_out = [torch.empty_like(self.wq, device="cpu").pin_memory(),
+                        torch.empty_like(self.xr, device="cpu").pin_memory()]
+        self.h2d = sum(t.numel() * t.element_size() for t in self.pin_in)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.pin_out)
+
+    def e2e_step(self):
+        self.w.copy_(self.pin_in[0], non_blocking=True)
+        self.x.copy_(self.pin_in[1], non_blocking=True)
+        self.step()
+        self.pin_out[0].copy_(self.wq, non_blocking=True)
+        self.pin_out[1].copy_(self.xr, non_blocking=True)
+
+    def oracle_rate(self, budget_s=10.0):
+        import oracle
+        oracle.lib()
+        perm, signs = inputs.rpbh_params(self.d)
+        h = self.d & -self.d
+        w = self.host[0].view(torch.int16).numpy().view(np.uint16)
+        cb = self.cb
+        done, t0, chunk = 0, time.perf_counter(), 32
+        while time.perf_counter() - t0 < budget_s and done + chunk <= self.rows:
+            p, n = oracle.rpbh_quantize(w[done:done + chunk], perm, signs, h, cb, self.bits, is_bf16=True)
+            oracle.rpbh_dequantize_rotated(p, n, chunk, self.d, self.bits, cb, out_bf16=True)
+            done += chunk
+        dt = time.perf_counter() - t0
+        return done * self.d / dt, f"first {done} weight rows quantized + dequantized (no activations), {dt:.1f} s"
+
+
+WORKLOADS = {
+    "kv": KVWorkload,
+    "longctx": LongContextWorkload,
+    "rpbh-llm": lambda dev: RPBHWorkload(dev),
+    "rpbh-dit": lambda dev: RPBHWorkload(dev, rows=12288, d=3072, xrows=4096, bits=3, seed=4),
+}
+
+
+# ---------------------------------------------------------------------------------------------
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_ours(args):
+    world, rank, local = dist_setup(args)
+    dev = torch.device("cuda", local)
+    wl = WORKLOADS[args.workload](dev)
+    # warm-up
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+    barrier(world)
+
+    # timed region: whole steps, plus per-kernel events on the launching (current) stream
+    ev = {}
+    launches = 0
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(args.steps):
+            launches += wl.step(ev)
+        end.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        # a second identical pass without per-kernel events gives the step time
+        torch.cuda.synchronize()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record()
+        for _ in range(args.steps):
+            wl.step()
+        e2.record()
+        torch.cuda.synchronize()
+        barrier(world)
+    ms_total = min(start.elapsed_time(end), s2.elapsed_time(e2))
+    ms_total = max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+    value = world * wl.units * args.steps / (ms_total / 1e3)
+
+    per_kernel = {}
+    for k in wl.kernels:
+        evs = ev.get(k, [])
+        durs = [evs[i].elapsed_time(evs[i + 1]) for i in range(0, len(evs), 2)]
+        avg_ms = sum(durs) / len(durs)
+        per_kernel[k] = {"avg_us": avg_ms * 1e3, "launches": len(durs),
+                         "gbs": wl.bytes_per_launch[k] / (avg_ms / 1e3) / 1e9}
+    dom = max(wl.kernels, key=lambda k: per_kernel[k]["avg_us"] * per_kernel[k]["launches"])
+    peak, peak_kind = measured_peaks()
+    achieved = per_kernel[dom]["gbs"]
+
+    # end to end through the same API with pinned host buffers
+    wl.e2e_setup()
+    for _ in range(max(1, args.warmup // 2)):
+        wl.e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(2, min(args.steps, 10))
+    es.record()
+    for _ in range(e2e_steps):
+        wl.e2e_step()
+    ee.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(es.elapsed_time(ee), world)
+    e2e_value = world * wl.units * e2e_steps / (e2e_ms / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, sample = wl.oracle_rate(args.cpu_seconds)
+        cpu = {"value": rate, "unit": wl.unit, "cores": 1, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "vectors_or_elements_per_step_per_gpu": wl.units,
+                       "io_dtype": "bf16", "l2": "inputs larger than L2; no kernel reads data written by "
+                       "the kernel just before it", "parallelism": f"replicas x{world} (no collective)"},
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic_bytes(dom),
+                         "algorithmic_bytes_per_launch": wl.bytes_per_launch[dom]},
+            "kernels": per_kernel,
+            "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": wl.h2d,
+                    "d2h_bytes_per_step": wl.d2h},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle, as it stands, on the host cores: the reference arm of this benchmark."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.lib()
+    dev = torch.device("cpu")
+    # build the workload's host data only (no device needed)
+    if args.workload == "kv":
+        k, _ = inputs.kv_cache()
+        src = k.reshape(-1, 128)
+        name, unit, metric = KVWorkload.name, KVWorkload.unit, KVWorkload.metric
+        bits = inputs.tq3_sign_bits()
+        chunk = args.ref_chunk
+
+        def step(i):
+            lo = (i * chunk) % (src.shape[0] - chunk)
+            p, n, s = oracle.tq3_encode(src[lo:lo + chunk], bits, is_bf16=True)
+            oracle.tq3_decode(p, n, s, bits, out_bf16=True)
+            return chunk
+    else:
+        raise SystemExit(f"--impl reference supports the default workload only, not {args.workload}")
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    units = 0
+    for i in range(args.steps):
+        units += step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = units / dt
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": name, "sample_vectors_per_step": chunk},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+                             "sample": f"{chunk} vectors of the K cache per step, encode + decode"},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="kv")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-chunk", type=int, default=2048)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * wq.h -- C ABI of libwq_b200.so: the TQ3 KV-cache codec and the OrbitQuant RPBH weight path
+ * on NVIDIA B200 (sm_100a).
+ *
+ * Sources. Every entry point restates an operation of one of two pages:
+ *   "tq3_core.py" (ComfyUI-TurboQuant): module docstring (format and algorithm), tq3_quantize,
+ *       tq3_dequantize, _fwht_inplace, _quantize_to_indices, _pack_3bit, _unpack_3bit,
+ *       tq3_memory_bytes.
+ *   "orbit_quant.py" (OrbitQuant weight-only backend): gaussian_lloyd_max, hadamard_block_size,
+ *       rpbh_forward, rpbh_inverse, _fwht, pack_codes, unpack_codes, _quantize_rows,
+ *       OrbitQuantizer.quantize_, _dequantize_rotated, dequantize, forward.
+ *
+ * Conventions shared by every call:
+ *   - Pointers named "device" are CUDA device memory owned by the caller. Pointers named "host"
+ *     are ordinary host memory read during the call (their contents are copied into the launch,
+ *     so the caller may reuse them as soon as the call returns).
+ *   - The library allocates no memory and never synchronises. Device work is enqueued on
+ *     `stream` (a cudaStream_t; NULL means the legacy default stream) and runs asynchronously.
+ *   - Arguments are validated before anything is enqueued; a call that returns an error has
+ *     enqueued nothing. Data VALUES are not validated (NaN/Inf give unspecified output).
+ *   - An empty problem (n_vec == 0, rows == 0) returns WQ_OK and enqueues nothing; its pointers
+ *     may then be NULL.
+ *   - Element types: WQ_F32 = IEEE binary32, WQ_BF16 = bfloat16 (raw 16-bit patterns).
+ *   - All arithmetic is fp32 in the order the pages give, except the two L2 norms, whose
+ *     squares are summed in fp64 and rounded once to fp32 after the square root.
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WQ_OK = 0,
+    WQ_ERR_NULL = -1,             /* a required pointer is NULL                                */
+    WQ_ERR_SHAPE = -2,            /* negative count, bad dimension, or d beyond the maximum     */
+    WQ_ERR_DTYPE = -3,            /* dtype code not one of wq_dtype                            */
+    WQ_ERR_ALIGN = -4,            /* a pointer is not aligned as its call requires             */
+    WQ_ERR_BITS = -5,             /* bits not in {2, 3, 4}                                      */
+    WQ_ERR_NOT_QUANTIZABLE = -6,  /* d & -d < 32: the page skips such layers                    */
+    WQ_ERR_CUDA = -7              /* the CUDA runtime reported an error at launch               */
+} wq_status;
+
+typedef enum { WQ_F32 = 0, WQ_BF16 = 1 } wq_dtype;
+
+/* Largest power-of-two block the RPBH rotation uses, and the page's floor for it
+ * ("orbit_quant.py", MIN_HADAMARD_BLOCK). */
+#define WQ_RPBH_MIN_BLOCK 32
+/* Largest RPBH input dimension d the kernels accept (one weight row is held on chip). */
+#define WQ_RPBH_MAX_D 32768
+
+/* ============================================================================================
+ * TQ3 ("tq3_core.py")
+ * A TQ3 record encodes one 128-element vector as 48 bytes of 3-bit indices plus an fp32 norm
+ * and an fp32 scale (56 bytes, 3.5 bits per value; module docstring). Records are stored as
+ * three arrays: packed[n_vec][48], norms[n_vec], scales[n_vec] (the dict tq3_quantize returns).
+ * A [..., D] tensor with D a multiple of 128 is n_vec = numel / 128 consecutive vectors.
+ * ============================================================================================ */
+
+/* tq3_encode -- tq3_quantize. For each vector: n = max(||x||_2, 1e-8); y = (x / n) * s with s
+ * the sign flips; y = FWHT_128(y) * fp32(1/sqrt(128)) (7 butterfly stages, h = 1..64);
+ * scale = max(max|y|, 1e-8); idx_i = #{j : B_j < y_i / scale} against TQ3_BOUNDARIES;
+ * indices packed 8 per 24-bit little-endian group (_pack_3bit).
+ *   x          device, n_vec x 128 elements of x_dtype, 16-byte aligned.
+ *   sign_mask  host, 4 words: bit i of the 128-bit little-endian mask is sign draw i
+ *              (1 -> +1, 0 -> -1), i.e. _generate_sign_flips(128, seed).
+ *   packed     device, n_vec x 48 bytes, 16-byte aligned.  norms, scales  device, n_vec fp32.
+ * Errors: WQ_ERR_NULL, WQ_ERR_SHAPE (n_vec < 0), WQ_ERR_DTYPE, WQ_ERR_ALIGN, WQ_ERR_CUDA. */
+wq_status tq3_encode(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
+                     uint8_t *packed, float *norms, float *scales, void *stream);
+
+/* tq3_decode -- tq3_dequantize. For each record: y_i = TQ3_CENTROIDS[idx_i] * scale;
+ * y = FWHT_128(y) * fp32(1/sqrt(128)); out_i = (y_i * s_i) * norm. With out_dtype = WQ_BF16
+ * the fp32 result is rounded once to nearest-even bf16.
+ *   packed device, n_vec x 48 bytes, 16-byte aligned.  norms, scales  device, n_vec fp32.
+ *   sign_mask host, as for tq3_encode.  out  device, n_vec x 128 of out_dtype, 16-byte aligned.
+ * Errors: as tq3_encode. */
+wq_status tq3_decode(const uint8_t *packed, const float *norms, const float *scales, int64_t n_vec,
+                     const uint32_t *sign_mask, void *out, int out_dtype, void *stream);
+
+/* tq3_compressed_bytes -- tq3_memory_bytes' compressed size for n_vec vectors: 56 * n_vec
+ * (-1 if n_vec < 0 or the product overflows). */
+int64_t tq3_compressed_bytes(int64_t n_vec);
+
+/* ============================================================================================
+ * RPBH ("orbit_quant.py")
+ * A weight W[rows][d] (out x in, row-major) is rotated row by row with the shared randomized
+ * permuted block-Hadamard R = blkdiag(H_h) D P, h = d & -d (hadamard_block_size):
+ * (R w)_j = FWHT_h-block( w[perm[j]] * signs[j] ) * fp32(h ** -0.5).
+ * perm is a permutation of 0..d-1 (int32, device) and signs are +-1 (int8, device), i.e.
+ * rpbh_params(d). Entries of perm outside 0..d-1 are not rejected; they are clamped so that no
+ * access leaves the row, and the output is then unspecified.
+ * Packed codes form one flat MSB-first bitstream over the row-major [rows][d] codes, zero padded
+ * to a multiple of 8 codes (pack_codes): rpbh_packed_bytes(rows, d, bits) bytes.
+ * ============================================================================================ */
+
+/* rpbh_quantize_weight -- _quantize_rows. For each row: w_rot = R w (fp32);
+ * rho = ||w_rot||_2; u_j = w_rot_j / (rho + 1e-10); code_j = #{k : e_k < u_j} with
+ * e_k = (c_k + c_{k+1}) / 2 over the scaled codebook; codes packed MSB-first; row_norms[r] = rho
+ * stored in w_dtype (OrbitQuantizer.quantize_ keeps the norms in the weight dtype).
+ *   W          device, rows x d of w_dtype, 16-byte aligned.
+ *   perm, signs device, d entries each.   bits  2, 3 or 4.
+ *   codebook   host, 2^bits ascending fp32 centroids, already scaled (wq_rpbh_codebook).
+ *   packed     device, rpbh_packed_bytes(rows, d, bits) bytes, 4-byte aligned.
+ *   row_norms  device, rows entries of w_dtype.
+ * Errors: WQ_ERR_NULL, WQ_ERR_SHAPE (rows < 0, d <= 0, d > WQ_RPBH_MAX_D or the row does not
+ * fit on chip), WQ_ERR_NOT_QUANTIZABLE (d & -d < 32), WQ_ERR_BITS, WQ_ERR_DTYPE, WQ_ERR_ALIGN,
+ * WQ_ERR_CUDA. */
+wq_status rpbh_quantize_weight(const void *W, int w_dtype, int64_t rows, int64_t d,
+                               const int32_t *perm, const int8_t *signs, int bits,
+                               const float *codebook, uint8_t *packed, void *row_norms,
+                               void *stream);
+
+/* rpbh_dequantize_weight -- _dequantize_rotated, and with unrotate = 1 dequantize.
+ * Rotated (unrotate = 0): out[r][j] = codebook[code] * row_norm[r] in out_dtype; for WQ_BF16 the
+ * page's bf16 product bf16(bf16(codebook[code]) * bf16(row_norm[r])).
+ * Unrotated (unrotate = 1): the fp32 rotated weight is mapped back with rpbh_inverse,
+ * z = FWHT_h-block(w') * fp32(h ** -0.5) * signs, out[r][perm[j]] = z[r][j]
+ * (the same as out[r][i] = z[r][inv_perm[i]]); WQ_BF16 output rounds that fp32 result once.
+ *   packed     device, as written by rpbh_quantize_weight, 4-byte aligned.
+ *   row_norms  device, rows entries of norm_dtype.  codebook  host, 2^bits fp32.
+ *   perm, signs device (read only when unrotate = 1; may be NULL otherwise).
+ *   out        device, rows x d of out_dtype, 16-byte aligned.
+ * Errors: as rpbh_quantize_weight. */
+wq_status rpbh_dequantize_weight(const uint8_t *packed, const void *row_norms, int norm_dtype,
+                                 int64_t rows, int64_t d, int bits, const float *codebook,
+                                 const int32_t *perm, const int8_t *signs, int unrotate,
+                                 void *out, int out_dtype, void *stream);
+
+/* rpbh_rotate_activations -- the activation side of OrbitQuantizer.forward: x_rot = R x per row,
+ * computed in fp32 and rounded once to the output dtype (the page runs the butterflies in the
+ * activation dtype; one final rounding is at least as accurate).
+ *   x, x_rot   device, rows x d of dtype, 16-byte aligned (x_rot may not alias x).
+ *   perm, signs device, d entries each.
+ * Errors: WQ_ERR_NULL, WQ_ERR_SHAPE, WQ_ERR_NOT_QUANTIZABLE, WQ_ERR_DTYPE, WQ_ERR_ALIGN,
+ * WQ_ERR_CUDA. */
+wq_status rpbh_rotate_activations(const void *x, int dtype, int64_t rows, int64_t d,
+                                  const int32_t *perm, const int8_t *signs, void *x_rot,
+                                  void *stream);
+
+/* rpbh_packed_bytes -- size of the packed bitstream: ceil(rows * d / 8) * bits (-1 on a bad
+ * argument). */
+int64_t rpbh_packed_bytes(int64_t rows, int64_t d, int bits);
+
+/* ============================================================================================
+ * Host helpers (run on the CPU, synchronous)
+ * ============================================================================================ */
+
+/* wq_gaussian_lloyd_max -- gaussian_lloyd_max: the 2^bits MSE-optimal levels for N(0,1),
+ * ascending. Initialised at sqrt(2) * erfinv(2q - 1), q = (k + 0.5) / 2^bits, then `iters`
+ * rounds of midpoint edges and conditional means (phi(lo) - phi(hi)) / (Phi(hi) - Phi(lo)),
+ * in fp64; the result is rounded once to fp32. `out` is host memory for 2^bits floats.
+ * Errors: WQ_ERR_NULL, WQ_ERR_BITS (bits outside 1..4), WQ_ERR_SHAPE (iters < 0). */
+wq_status wq_gaussian_lloyd_max(int bits, int iters, float *out);
+
+/* wq_rpbh_codebook -- the codebook OrbitQuantizer.quantize_ stores for input dimension d:
+ * fp32(gaussian_lloyd_max(bits, 200)) * fp32(d ** -0.5). `out` host, 2^bits floats.
+ * Errors: WQ_ERR_NULL, WQ_ERR_BITS, WQ_ERR_SHAPE (d <= 0). */
+wq_status wq_rpbh_codebook(int bits, int64_t d, float *out);
+
+/* wq_status_string -- a static, NUL-terminated description of a status code. */
+const char *wq_status_string(int status);
+
+/* wq_version -- library version, (major << 16) | minor. */
+int wq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WQ_H */

@@ -1,0 +1,123 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol the
+header declares, rejects bad arguments with the documented status codes before touching the
+device, and its host helpers agree with the oracle."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+from conftest import ROOT
+from weight_quantization_b200 import inputs
+
+WQ_OK, WQ_ERR_NULL, WQ_ERR_SHAPE, WQ_ERR_DTYPE, WQ_ERR_ALIGN, WQ_ERR_BITS, WQ_ERR_NOT_QUANTIZABLE = 0, -1, -2, -3, -4, -5, -6
+
+
+@pytest.fixture(scope="module")
+def wq():
+    from weight_quantization_b200 import build, ops
+    build.build()
+    return ops
+
+
+def header_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_declared_symbol(wq):
+    names = header_functions()
+    assert len(names) >= 11, names
+    L = C.CDLL(wq.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+    assert set(names) <= set(wq.PROTOTYPES), set(names) - set(wq.PROTOTYPES)
+
+
+def test_version_and_status_strings(wq):
+    L = wq.lib()
+    assert L.wq_version() >= 1
+    for st in range(-7, 1):
+        assert L.wq_status_string(st)
+    assert L.wq_status_string(99) == b"unknown status"
+
+
+def test_tq3_argument_validation(wq):
+    L = wq.lib()
+    m = np.zeros(4, np.uint32)
+    mp = m.ctypes.data
+    A = 0x10000  # a 16-byte aligned fake device address: validation fails before any use
+    assert L.tq3_encode(A, 1, 0, mp, A, A, A, None) == WQ_OK          # empty: nothing enqueued
+    assert L.tq3_encode(None, 1, 0, None, None, None, None, None) == WQ_OK
+    assert L.tq3_encode(A, 1, -1, mp, A, A, A, None) == WQ_ERR_SHAPE
+    assert L.tq3_encode(A, 7, 4, mp, A, A, A, None) == WQ_ERR_DTYPE
+    assert L.tq3_encode(None, 1, 4, mp, A, A, A, None) == WQ_ERR_NULL
+    assert L.tq3_encode(A, 1, 4, None, A, A, A, None) == WQ_ERR_NULL
+    assert L.tq3_encode(A + 8, 1, 4, mp, A, A, A, None) == WQ_ERR_ALIGN
+    assert L.tq3_encode(A, 1, 4, mp, A + 4, A, A, None) == WQ_ERR_ALIGN
+    assert L.tq3_encode(A, 1, 4, mp, A, A + 2, A, None) == WQ_ERR_ALIGN
+    assert L.tq3_decode(A, A, A, 0, mp, A, 0, None) == WQ_OK
+    assert L.tq3_decode(A, A, A, -3, mp, A, 0, None) == WQ_ERR_SHAPE
+    assert L.tq3_decode(A, A, A, 3, mp, A, 5, None) == WQ_ERR_DTYPE
+    assert L.tq3_decode(A, None, A, 3, mp, A, 0, None) == WQ_ERR_NULL
+    assert L.tq3_decode(A, A, A, 3, mp, A + 4, 0, None) == WQ_ERR_ALIGN
+    assert L.tq3_compressed_bytes(10) == 560
+    assert L.tq3_compressed_bytes(-1) == -1
+
+
+def test_rpbh_argument_validation(wq):
+    L = wq.lib()
+    cb = np.zeros(16, np.float32).ctypes.data
+    A = 0x10000
+    q = lambda W=A, dt=1, rows=4, d=3072, perm=A, signs=A, bits=3, cbp=cb, packed=A, norms=A: \
+        L.rpbh_quantize_weight(W, dt, rows, d, perm, signs, bits, cbp, packed, norms, None)
+    assert q(rows=0) == WQ_OK
+    assert q(rows=-1) == WQ_ERR_SHAPE
+    assert q(d=0) == WQ_ERR_SHAPE
+    assert q(d=100) == WQ_ERR_NOT_QUANTIZABLE     # 100 & -100 = 4 < 32
+    assert q(d=48) == WQ_ERR_NOT_QUANTIZABLE      # 16 < 32
+    assert q(d=WQ_MAX_D * 2) == WQ_ERR_SHAPE
+    assert q(bits=1) == WQ_ERR_BITS and q(bits=5) == WQ_ERR_BITS
+    assert q(dt=3) == WQ_ERR_DTYPE
+    assert q(W=None) == WQ_ERR_NULL and q(cbp=None) == WQ_ERR_NULL and q(norms=None) == WQ_ERR_NULL
+    assert q(W=A + 8) == WQ_ERR_ALIGN and q(packed=A + 2) == WQ_ERR_ALIGN
+    dq = lambda unrot=1, perm=A, signs=A, bits=3, nd=1, od=0, out=A, d=3072: \
+        L.rpbh_dequantize_weight(A, A, nd, 4, d, bits, cb, perm, signs, unrot, out, od, None)
+    assert dq(perm=None) == WQ_ERR_NULL
+    assert dq(bits=6) == WQ_ERR_BITS
+    assert dq(od=9) == WQ_ERR_DTYPE
+    assert dq(out=A + 4) == WQ_ERR_ALIGN
+    assert dq(d=96 + 8) == WQ_ERR_NOT_QUANTIZABLE
+    r = lambda x=A, d=3072, dt=1: L.rpbh_rotate_activations(x, dt, 4, d, A, A, A, None)
+    assert r(x=None) == WQ_ERR_NULL and r(d=40) == WQ_ERR_NOT_QUANTIZABLE and r(dt=2) == WQ_ERR_DTYPE
+    assert L.rpbh_packed_bytes(4096, 11008, 3) == 4096 * 11008 * 3 // 8
+    assert L.rpbh_packed_bytes(1, 5, 3) == 3 and L.rpbh_packed_bytes(-1, 5, 3) == -1
+
+
+WQ_MAX_D = 32768
+
+
+def test_lloyd_max_host_helper_matches_oracle(wq, oracle):
+    for bits in (1, 2, 3, 4):
+        assert np.array_equal(wq.gaussian_lloyd_max(bits), oracle.gaussian_lloyd_max(bits))
+    for bits in (2, 3, 4):
+        for d in (32, 96, 3072, 11008):
+            assert np.array_equal(wq.rpbh_codebook(bits, d), oracle.rpbh_codebook(bits, d))
+    with pytest.raises(wq.WQError):
+        wq.gaussian_lloyd_max(5)
+    with pytest.raises(wq.WQError):
+        wq.rpbh_codebook(3, 0)
+
+
+def test_sign_mask_layout(wq):
+    bits = inputs.tq3_sign_bits()
+    m = wq.sign_mask_words(bits)
+    assert np.array_equal(m, inputs.tq3_sign_mask_words(bits))
+    assert [hex(v) for v in m] == ["0x3fd74222", "0x1ab7c17", "0xff4abaf6", "0x656b5fe7"]

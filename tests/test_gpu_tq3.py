@@ -1,0 +1,155 @@
+"""GPU parity of the TQ3 kernels against the oracle, through the C ABI (page "tq3_core.py")."""
+import numpy as np
+import pytest
+import torch
+
+import parity
+from weight_quantization_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+BITS = inputs.tq3_sign_bits()
+
+
+@pytest.fixture(scope="module")
+def wq():
+    from weight_quantization_b200 import build, ops
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return ops
+
+
+@pytest.fixture(scope="module")
+def mask(wq):
+    return wq.sign_mask_words(BITS)
+
+
+def _encode(wq, x_np, is_bf16, mask):
+    t = torch.from_numpy(x_np.view(np.int16) if is_bf16 else x_np)
+    t = t.view(torch.bfloat16) if is_bf16 else t
+    p, n, s = wq.tq3_encode(t.cuda(), mask)
+    torch.cuda.synchronize()
+    return p.cpu().numpy(), n.cpu().numpy(), s.cpu().numpy()
+
+
+def test_encode_roundtrip_config_fp32(wq, oracle, mask):
+    """4096 x 128 fp32: 4064 N(0,1) vectors and 32 constant blocks (value 1.0)."""
+    x = inputs.tq3_roundtrip()
+    p, n, s = _encode(wq, x, False, mask)
+    st = parity.check_tq3_encode(oracle, x, BITS, False, p, n, s)
+    # every constant block has 11 exact-zero coefficients; they are exact ties at boundary 0.0
+    assert st["exact_zero_coeffs"] >= 352
+    print("tq3 encode C1", st)
+
+
+@pytest.mark.parametrize("n_vec", [1, 3, 33, 127, 128, 129, 1000])
+@pytest.mark.parametrize("is_bf16", [False, True])
+def test_encode_ragged(wq, oracle, mask, n_vec, is_bf16):
+    x = inputs.gaussian((n_vec, 128), seed=1000 + n_vec) * 4
+    if is_bf16:
+        x = inputs.to_bf16_bits(torch.from_numpy(x))
+    p, n, s = _encode(wq, x, is_bf16, mask)
+    parity.check_tq3_encode(oracle, x, BITS, is_bf16, p, n, s)
+
+
+def test_encode_degenerate_vectors(wq, oracle, mask):
+    rows = [np.zeros(128), np.full(128, 1.0), np.full(128, 2.5), np.full(128, -3.0),
+            np.full(128, 1e-30), np.full(128, 1e30), np.eye(128)[5] * 7.0, np.eye(128)[0] * -1e-3,
+            np.where(np.arange(128) % 2 == 0, 1.0, -1.0), np.linspace(-1, 1, 128),
+            np.sin(np.linspace(0, 2 * np.pi, 128)), np.r_[np.zeros(127), 40.0]]
+    x = np.array(rows, np.float32)
+    p, n, s = _encode(wq, x, False, mask)
+    st = parity.check_tq3_encode(oracle, x, BITS, False, p, n, s)
+    assert st["bytes_equal"]
+    assert n[0] == np.float32(1e-8) and s[0] == np.float32(1e-8)
+    assert p[0].tobytes() == bytes.fromhex("dbb66d") * 16
+
+
+def test_encode_kv_cache_full_size(wq, oracle, mask):
+    """K and V caches [8, 8, 4096, 128] bf16 = 524,288 vectors, every vector checked."""
+    k, v = inputs.kv_cache()
+    total = {"vectors": 0, "index_mismatches": 0, "coeffs_in_tie_window": 0, "norms_equal": 0}
+    for name, t in (("K", k), ("V", v)):
+        x = t.reshape(-1, 128)
+        p, n, s = _encode(wq, x, True, mask)
+        st = parity.check_tq3_encode(oracle, x, BITS, True, p, n, s)
+        for key in total:
+            total[key] += st[key]
+    assert total["vectors"] == 524288
+    print("tq3 encode C2", total)
+
+
+@pytest.mark.parametrize("out_bf16", [False, True])
+def test_decode_roundtrip_config(wq, oracle, mask, out_bf16):
+    x = inputs.tq3_roundtrip()
+    packed, norms, scales = oracle.tq3_encode(x, BITS)
+    out = wq.tq3_decode(torch.from_numpy(packed).cuda(), torch.from_numpy(norms).cuda(),
+                        torch.from_numpy(scales).cuda(), mask,
+                        out_dtype=torch.bfloat16 if out_bf16 else torch.float32)
+    g = out.cpu()
+    g = g.view(torch.int16).numpy().view(np.uint16) if out_bf16 else g.numpy()
+    st = parity.check_tq3_decode(oracle, packed, norms, scales, BITS, g, out_bf16)
+    print("tq3 decode C1", out_bf16, st)
+
+
+@pytest.mark.parametrize("n_vec", [1, 5, 129, 777])
+def test_decode_ragged(wq, oracle, mask, n_vec):
+    idx = inputs.uniform_int((n_vec, 128), 8, seed=n_vec)
+    packed = oracle.tq3_pack(idx)
+    norms = (np.abs(inputs.gaussian((n_vec,), seed=n_vec + 1)) * 3 + 0.1).astype(np.float32)
+    scales = (np.abs(inputs.gaussian((n_vec,), seed=n_vec + 2)) * 0.2 + 0.05).astype(np.float32)
+    out = wq.tq3_decode(torch.from_numpy(packed).cuda(), torch.from_numpy(norms).cuda(),
+                        torch.from_numpy(scales).cuda(), mask).cpu().numpy()
+    parity.check_tq3_decode(oracle, packed, norms, scales, BITS, out, False)
+
+
+def test_decode_long_context_full_size(wq, oracle, mask):
+    """1,048,576 records decoded to bf16 [1, 8, 131072, 128]; a strided sample plus the tail
+    checked against the oracle, every output checked for finiteness."""
+    packed, norms, scales = inputs.long_context_records()
+    out = wq.tq3_decode(torch.from_numpy(packed).cuda(), torch.from_numpy(norms).cuda(),
+                        torch.from_numpy(scales).cuda(), mask, out_dtype=torch.bfloat16)
+    assert bool(torch.isfinite(out.float()).all())
+    n = packed.shape[0]
+    sel = np.unique(np.concatenate([np.arange(0, n, 37), np.arange(n - 300, n)]))
+    g = out[torch.from_numpy(sel).cuda()].cpu().view(torch.int16).numpy().view(np.uint16)
+    st = parity.check_tq3_decode(oracle, packed[sel], norms[sel], scales[sel], BITS, g, True)
+    print("tq3 decode C3 sample", st)
+
+
+def test_roundtrip_quality_on_gpu(wq, mask):
+    """The page's quality bar (mean cosine > 0.97) holds for the GPU round trip."""
+    x = torch.from_numpy(inputs.tq3_roundtrip()).cuda()
+    p, n, s = wq.tq3_encode(x, mask)
+    xr = wq.tq3_decode(p, n, s, mask)
+    cos = torch.nn.functional.cosine_similarity(x.double(), xr.double(), dim=-1)
+    assert cos[:4064].mean().item() > 0.97
+    assert cos[4064:].min().item() > 0.97
+
+
+def test_outputs_stay_in_bounds_and_streams(wq, oracle, mask):
+    """Canaries after the last record stay untouched; work runs on the caller's stream."""
+    n_vec = 77
+    x = torch.from_numpy(inputs.gaussian((n_vec, 128), seed=9)).cuda()
+    packed = torch.full((n_vec + 3, 48), 0xAB, dtype=torch.uint8, device="cuda")
+    norms = torch.full((n_vec + 5,), -7.0, device="cuda")
+    scales = torch.full((n_vec + 5,), -7.0, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        wq.tq3_encode(x, mask, packed=packed[:n_vec], norms=norms[:n_vec], scales=scales[:n_vec])
+        out = torch.full((n_vec + 2, 128), -9.0, device="cuda")
+        wq.tq3_decode(packed[:n_vec], norms[:n_vec], scales[:n_vec], mask, out=out[:n_vec])
+    s.synchronize()
+    assert bool((packed[n_vec:] == 0xAB).all()) and bool((norms[n_vec:] == -7).all())
+    assert bool((scales[n_vec:] == -7).all()) and bool((out[n_vec:] == -9).all())
+    parity.check_tq3_encode(oracle, x.cpu().numpy(), BITS, False, packed[:n_vec].cpu().numpy(),
+                            norms[:n_vec].cpu().numpy(), scales[:n_vec].cpu().numpy())
+
+
+def test_empty_and_errors(wq, mask):
+    x = torch.empty(0, 128, device="cuda")
+    p, n, s = wq.tq3_encode(x, mask)
+    assert p.shape == (0, 1, 48)
+    with pytest.raises(wq.WQError):
+        wq.tq3_encode(torch.zeros(4, 128, device="cuda", dtype=torch.float32)[:, :128], mask,
+                      packed=torch.empty(4 * 48 + 1, dtype=torch.uint8, device="cuda")[1:].view(4, 1, 48))

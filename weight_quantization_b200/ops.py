@@ -1,0 +1,207 @@
+"""Thin Python binding of libwq_b200.so (argument marshalling only).
+
+Every function here checks tensor placement, dtype and contiguity, allocates outputs with torch
+when the caller does not pass them, and forwards raw pointers, sizes and the current CUDA stream
+to the C ABI declared in include/wq.h. All compute happens in the library's CUDA kernels; there
+is no CPU or PyTorch fallback, and a missing library raises at the first call.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwq_b200.so")
+
+WQ_F32, WQ_BF16 = 0, 1
+_DT = {torch.float32: WQ_F32, torch.bfloat16: WQ_BF16}
+
+# C prototypes of include/wq.h: name -> (restype, argtypes)
+_vp, _i64, _int = C.c_void_p, C.c_int64, C.c_int
+PROTOTYPES = {
+    "tq3_encode": (_int, [_vp, _int, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "tq3_decode": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _int, _vp]),
+    "tq3_compressed_bytes": (_i64, [_i64]),
+    "rpbh_quantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp]),
+    "rpbh_dequantize_weight": (_int, [_vp, _vp, _int, _i64, _i64, _int, _vp, _vp, _vp, _int, _vp, _int, _vp]),
+    "rpbh_rotate_activations": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "rpbh_packed_bytes": (_i64, [_i64, _i64, _int]),
+    "wq_gaussian_lloyd_max": (_int, [_int, _int, _vp]),
+    "wq_rpbh_codebook": (_int, [_int, _i64, _vp]),
+    "wq_status_string": (C.c_char_p, [_int]),
+    "wq_version": (_int, []),
+}
+
+_lib = None
+
+
+class WQError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {lib().wq_status_string(status).decode()} (status {status})")
+        self.status = status
+
+
+def lib():
+    """Load the CUDA library (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libwq_b200.so not found at {LIB_PATH}: build it with "
+                               "`python -m weight_quantization_b200.build` (there is no fallback)")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in PROTOTYPES.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise WQError(fn, status)
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def sign_mask_words(sign_bits) -> np.ndarray:
+    """Lay out 128 sign draws (1 = +1, 0 = -1) as the four host words the ABI takes."""
+    bits = np.asarray(sign_bits, dtype=np.uint64).reshape(4, 32)
+    return (bits << np.arange(32, dtype=np.uint64)).sum(axis=1).astype(np.uint32)
+
+
+def _mask_arg(mask) -> np.ndarray:
+    m = np.ascontiguousarray(np.asarray(mask, dtype=np.uint32))
+    if m.shape != (4,):
+        raise ValueError("sign mask must be 4 uint32 words")
+    return m
+
+
+# ---------------------------------------------------------------------------------------------
+# TQ3
+# ---------------------------------------------------------------------------------------------
+def tq3_encode(x: torch.Tensor, sign_mask, packed=None, norms=None, scales=None):
+    """TQ3-encode a [..., D] fp32/bf16 CUDA tensor (D a multiple of 128).
+
+    Returns (packed uint8 [..., D/128, 48], norms fp32 [..., D/128], scales fp32 [..., D/128]).
+    """
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32 or bfloat16")
+    if x.ndim == 0 or x.shape[-1] % 128 != 0 or x.shape[-1] <= 0:
+        raise ValueError("last dim must be a positive multiple of 128")
+    lead = tuple(x.shape[:-1]) + (x.shape[-1] // 128,)
+    n_vec = x.numel() // 128
+    if packed is None:
+        packed = torch.empty(lead + (48,), dtype=torch.uint8, device=x.device)
+    if norms is None:
+        norms = torch.empty(lead, dtype=torch.float32, device=x.device)
+    if scales is None:
+        scales = torch.empty(lead, dtype=torch.float32, device=x.device)
+    m = _mask_arg(sign_mask)
+    st = lib().tq3_encode(_dev(x, "x"), _DT[x.dtype], n_vec, m.ctypes.data, _dev(packed, "packed"),
+                          _dev(norms, "norms"), _dev(scales, "scales"), _stream(x.device))
+    _check("tq3_encode", st)
+    return packed, norms, scales
+
+
+def tq3_decode(packed: torch.Tensor, norms: torch.Tensor, scales: torch.Tensor, sign_mask,
+               out_dtype=torch.float32, out=None):
+    """Decode TQ3 records back to [..., 128] values of out_dtype (fp32 or bf16)."""
+    if packed.shape[-1] != 48 or tuple(packed.shape[:-1]) != tuple(norms.shape) or norms.shape != scales.shape:
+        raise ValueError("packed must be [..., 48] with norms/scales of shape [...]")
+    n_vec = norms.numel()
+    if out is None:
+        out = torch.empty(tuple(norms.shape) + (128,), dtype=out_dtype, device=packed.device)
+    m = _mask_arg(sign_mask)
+    st = lib().tq3_decode(_dev(packed, "packed"), _dev(norms, "norms"), _dev(scales, "scales"), n_vec,
+                          m.ctypes.data, _dev(out, "out"), _DT[out.dtype], _stream(packed.device))
+    _check("tq3_decode", st)
+    return out
+
+
+def tq3_compressed_bytes(n_vec: int) -> int:
+    return int(lib().tq3_compressed_bytes(n_vec))
+
+
+# ---------------------------------------------------------------------------------------------
+# RPBH
+# ---------------------------------------------------------------------------------------------
+def _codebook_arg(codebook, bits) -> np.ndarray:
+    cb = np.ascontiguousarray(np.asarray(codebook, dtype=np.float32))
+    if cb.shape != (1 << bits,):
+        raise ValueError(f"codebook must hold {1 << bits} floats")
+    return cb
+
+
+def rpbh_packed_bytes(rows: int, d: int, bits: int) -> int:
+    return int(lib().rpbh_packed_bytes(rows, d, bits))
+
+
+def rpbh_quantize_weight(W: torch.Tensor, perm: torch.Tensor, signs: torch.Tensor, bits: int, codebook,
+                         packed=None, row_norms=None):
+    """Quantize W [rows, d] (fp32/bf16). Returns (packed uint8 bitstream, row_norms in W's dtype)."""
+    rows, d = W.shape
+    cb = _codebook_arg(codebook, bits)
+    if packed is None:
+        packed = torch.empty(max(rpbh_packed_bytes(rows, d, bits), 0), dtype=torch.uint8, device=W.device)
+    if row_norms is None:
+        row_norms = torch.empty(rows, dtype=W.dtype, device=W.device)
+    st = lib().rpbh_quantize_weight(_dev(W, "W"), _DT.get(W.dtype, -1), rows, d, _dev(perm, "perm"),
+                                    _dev(signs, "signs"), bits, cb.ctypes.data, _dev(packed, "packed"),
+                                    _dev(row_norms, "row_norms"), _stream(W.device))
+    _check("rpbh_quantize_weight", st)
+    return packed, row_norms
+
+
+def rpbh_dequantize_weight(packed: torch.Tensor, row_norms: torch.Tensor, rows: int, d: int, bits: int, codebook,
+                           perm=None, signs=None, unrotate: bool = False, out_dtype=torch.float32, out=None):
+    """Dequantize to [rows, d]: the rotated weight W P^T, or (unrotate=True) W itself."""
+    cb = _codebook_arg(codebook, bits)
+    if out is None:
+        out = torch.empty(rows, d, dtype=out_dtype, device=packed.device)
+    pp = _dev(perm, "perm") if perm is not None else None
+    sp = _dev(signs, "signs") if signs is not None else None
+    st = lib().rpbh_dequantize_weight(_dev(packed, "packed"), _dev(row_norms, "row_norms"),
+                                      _DT.get(row_norms.dtype, -1), rows, d, bits, cb.ctypes.data, pp, sp,
+                                      int(bool(unrotate)), _dev(out, "out"), _DT.get(out.dtype, -1),
+                                      _stream(packed.device))
+    _check("rpbh_dequantize_weight", st)
+    return out
+
+
+def rpbh_rotate_activations(x: torch.Tensor, perm: torch.Tensor, signs: torch.Tensor, out=None):
+    """x_rot = blkdiag(H_h) D P x for every row of x [rows, d] (fp32/bf16)."""
+    rows, d = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    st = lib().rpbh_rotate_activations(_dev(x, "x"), _DT.get(x.dtype, -1), rows, d, _dev(perm, "perm"),
+                                       _dev(signs, "signs"), _dev(out, "out"), _stream(x.device))
+    _check("rpbh_rotate_activations", st)
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# host helpers
+# ---------------------------------------------------------------------------------------------
+def gaussian_lloyd_max(bits: int, iters: int = 200) -> np.ndarray:
+    out = np.zeros(1 << bits, np.float32)
+    _check("wq_gaussian_lloyd_max", lib().wq_gaussian_lloyd_max(bits, iters, out.ctypes.data))
+    return out
+
+
+def rpbh_codebook(bits: int, d: int) -> np.ndarray:
+    out = np.zeros(1 << bits, np.float32)
+    _check("wq_rpbh_codebook", lib().wq_rpbh_codebook(bits, d, out.ctypes.data))
+    return out
