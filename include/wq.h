@@ -161,6 +161,12 @@ wq_status wq_gaussian_lloyd_max(int bits, int iters, float *out);
  * Errors: WQ_ERR_NULL, WQ_ERR_BITS, WQ_ERR_SHAPE (d <= 0). */
 wq_status wq_rpbh_codebook(int bits, int64_t d, float *out);
 
+/* wq_device_fault -- reads and clears the library's sticky device fault bits. A TMA kernel whose
+ * bounded wait for its tile transfer runs out (which does not happen in normal operation) sets
+ * bit 0 and returns early, leaving its outputs unspecified. Synchronous (a device-to-host copy on
+ * the legacy default stream); `flags` is host memory. Errors: WQ_ERR_NULL, WQ_ERR_CUDA. */
+wq_status wq_device_fault(unsigned int *flags);
+
 /* wq_status_string -- a static, NUL-terminated description of a status code. */
 const char *wq_status_string(int status);
 

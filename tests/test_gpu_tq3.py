@@ -121,7 +121,7 @@ def test_roundtrip_quality_on_gpu(wq, mask):
     """The page's quality bar (mean cosine > 0.97) holds for the GPU round trip."""
     x = torch.from_numpy(inputs.tq3_roundtrip()).cuda()
     p, n, s = wq.tq3_encode(x, mask)
-    xr = wq.tq3_decode(p, n, s, mask)
+    xr = wq.tq3_decode(p, n, s, mask).reshape(x.shape)
     cos = torch.nn.functional.cosine_similarity(x.double(), xr.double(), dim=-1)
     assert cos[:4064].mean().item() > 0.97
     assert cos[4064:].min().item() > 0.97
@@ -153,3 +153,47 @@ def test_empty_and_errors(wq, mask):
     with pytest.raises(wq.WQError):
         wq.tq3_encode(torch.zeros(4, 128, device="cuda", dtype=torch.float32)[:, :128], mask,
                       packed=torch.empty(4 * 48 + 1, dtype=torch.uint8, device="cuda")[1:].view(4, 1, 48))
+
+
+@pytest.mark.parametrize("table", ["seed7", "all_plus", "all_minus"])
+@pytest.mark.parametrize("is_bf16", [False, True])
+def test_other_sign_tables(wq, oracle, table, is_bf16):
+    """Sign tables other than the page's seed-42 draws take the runtime-mask kernels."""
+    bits = {"seed7": inputs.tq3_sign_bits(7), "all_plus": np.ones(128, np.uint8),
+            "all_minus": np.zeros(128, np.uint8)}[table]
+    m = wq.sign_mask_words(bits)
+    x = inputs.gaussian((300, 128), seed=77) * 3
+    x[5] = 2.5  # a constant block
+    if is_bf16:
+        x = inputs.to_bf16_bits(torch.from_numpy(x))
+    t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16) if is_bf16 else torch.from_numpy(x)
+    p, n, s = wq.tq3_encode(t.cuda(), m)
+    parity.check_tq3_encode(oracle, x, bits, is_bf16, p.cpu().numpy(), n.cpu().numpy(), s.cpu().numpy())
+    for out_dtype in (torch.float32, torch.bfloat16):
+        out = wq.tq3_decode(p, n, s, m, out_dtype=out_dtype).cpu()
+        g = out.view(torch.int16).numpy().view(np.uint16) if out_dtype == torch.bfloat16 else out.numpy()
+        st = parity.check_tq3_decode(oracle, p.cpu().numpy().reshape(-1, 48), n.cpu().numpy().ravel(),
+                                     s.cpu().numpy().ravel(), bits, g, out_dtype == torch.bfloat16)
+        assert st["bit_exact"]
+
+
+def test_extreme_dynamic_range(wq, oracle, mask):
+    """Vectors spanning many binades (down to subnormal quotients) still match the oracle's IEEE
+    divisions bit for bit."""
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((2000, 128)) * np.exp(rng.uniform(-40, 40, (2000, 128)))).astype(np.float32)
+    x[:20, :64] = 1e-40  # subnormal inputs next to normal ones
+    x[20:40] = np.float32(3e-39)
+    x[40:60, 0] = 3e38
+    p, n, s = _encode(wq, x, False, mask)
+    st = parity.check_tq3_encode(oracle, x, BITS, False, p, n, s)
+    assert st["bytes_equal"] and st["norms_equal"] == x.shape[0]
+    xb = inputs.to_bf16_bits(torch.from_numpy(x))
+    p, n, s = _encode(wq, xb, True, mask)
+    st = parity.check_tq3_encode(oracle, xb, BITS, True, p, n, s)
+    assert st["bytes_equal"]
+
+
+def test_no_device_fault_recorded(wq):
+    torch.cuda.synchronize()
+    assert wq.device_fault() == 0

@@ -1,14 +1,23 @@
 // TQ3 KV-cache codec on sm_100a: page "tq3_core.py" (tq3_quantize, tq3_dequantize).
 //
-// Layout: one thread owns one 128-element vector for the whole transform. The 128 values live in
-// registers, so the 7 butterfly stages of the FWHT need no shuffles and no shared memory, every
-// element index is a compile-time constant, and the per-vector scalars (norm, reciprocal, scale)
-// are computed once per vector rather than once per lane.
+// Layout: two threads own one 128-element vector. Lanes 0-15 of a warp hold elements 0..63 of 16
+// vectors and lanes 16-31 hold elements 64..127 of the same vectors, so six of the seven FWHT
+// stages run in registers and only the last one (h = 64) exchanges values with a shuffle. A CTA of
+// 128 threads handles 64 vectors. The encoder's input tile is loaded from HBM by TMA into shared
+// memory with 128-byte swizzling; the decoder stages its output tile in the same swizzled layout
+// and writes it back with coalesced 16-byte stores. Either way every thread reads or writes its
+// own 128-byte row segment without bank conflicts and global traffic is whole, contiguous tiles.
 //
-// Rounding follows the page step by step in fp32 (the library is built with -fmad=false, so no
-// multiply is fused into a following add), which makes the packed bytes reproducible bit for
-// bit by any IEEE implementation of the same steps. The one reading the page leaves open is
-// the L2 norm's reduction: squares are summed in fp64 and the fp64 square root is rounded once.
+// Rounding follows the page step by step in fp32 (the library is built with -fmad=false; fused
+// operations are written explicitly only where they are exact), so packed bytes, norms and scales
+// are reproducible bit for bit:
+//   * the L2 norm sums exact fp64 squares and rounds the fp64 square root once to fp32;
+//   * x / n and xh / scale are correctly rounded quotients computed with Markstein's method: with
+//     r = RN(1/d), q0 = RN(x r), e = x - q0 d (exact by FMA), RN(q0 + e r) = RN(x / d)
+//     (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000 processor",
+//     IBM J. Res. Dev. 34(1), 1990); it is checked bit for bit against IEEE division by the tests;
+//   * the butterflies and post-multipliers are single IEEE additions and multiplications.
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -19,190 +28,360 @@ namespace wq {
 namespace tq3 {
 
 constexpr int kD = 128;
-constexpr int kThreads = 128;
+constexpr int kRows = 64;       // vectors per CTA
+constexpr int kThreads = 128;   // two threads per vector
+constexpr int kBoxBytes = kRows * 128;
+constexpr uint32_t kMaxPolls = 1u << 24;
+constexpr int64_t kMaxChunk = int64_t(1) << 30;  // vectors per launch (TMA row coordinates are int32)
 
-// TQ3_CENTROIDS (positive half; the negative half is its exact mirror) and TQ3_BOUNDARIES as
-// printed on the page, rounded to fp32 like torch.tensor(..., dtype=float32).
+// Set (sticky) by a kernel whose bounded wait for its TMA tile ran out; read by wq_device_fault.
+__device__ unsigned int g_fault;
+
+struct SignMask {
+    uint32_t w[4];  // bit i = sign draw i (1 -> +1, 0 -> -1)
+};
+
+// The draws of _generate_sign_flips(128, seed=42): the page's fixed table. Kernels specialised on it
+// fold the flips into compile-time constants; any other table takes the runtime path.
+__host__ __device__ constexpr uint32_t default_mask_word(int w) {
+    return w == 0 ? 0x3fd74222u : w == 1 ? 0x01ab7c17u : w == 2 ? 0xff4abaf6u : 0x656b5fe7u;
+}
+__host__ __device__ constexpr uint32_t default_flip(int e) {
+    return ((default_mask_word(e >> 5) >> (e & 31)) & 1u) ? 0u : 0x80000000u;
+}
+
+// Sign-bit XOR pattern for the pair of elements (e, e + 1), e = 64 * half + 2k, laid out like a
+// bf16x2 word (bit 15 = element e, bit 31 = element e + 1). H is all ones for half 1.
+template <bool kDefault>
+__device__ __forceinline__ uint32_t pair_flip(int k, uint32_t H, uint32_t mlo, uint32_t mhi) {
+    if (kDefault) {
+        const uint32_t c0 = (default_flip(2 * k) >> 16) | default_flip(2 * k + 1);
+        const uint32_t c1 = (default_flip(64 + 2 * k) >> 16) | default_flip(64 + 2 * k + 1);
+        return c0 ^ (H & (c0 ^ c1));
+    } else {
+        const uint32_t word = k < 16 ? mlo : mhi;
+        const uint32_t b = (~word >> ((2 * k) & 31)) & 3u;
+        return ((b & 1u) << 15) | ((b & 2u) << 30);
+    }
+}
+
+// fp32(1.0 / math.sqrt(128)), the post-multiplier of _fwht_inplace.
+__device__ __forceinline__ float fwht_post() { return __uint_as_float(0x3DB504F3u); }
+
+// Correctly rounded x / d given r = RN(1/d) (Markstein), two lanes at a time.
+__device__ __forceinline__ f32x2 div2(f32x2 x, f32x2 r, f32x2 neg_d) {
+    const f32x2 q0 = mul2(x, r);
+    const f32x2 e = fma2(q0, neg_d, x);
+    return fma2(e, r, q0);
+}
+
+// searchsorted(TQ3_BOUNDARIES, q, right=False) as a sum of exact 0/1 steps [q > B_j] computed on
+// the FMA pipe: for |B_j| >= 0.2304 any fp32 q above B_j exceeds it by at least 2^-26, so
+// (q - B_j) * 2^26 >= 1 and the saturated value is exactly 1; q <= B_j saturates to 0. The step at
+// B = 0 scales twice so that the smallest subnormal q > 0 still reaches 1.
+__device__ __forceinline__ float bucket_steps(float q) {
+    const float M = 67108864.0f;  // 2^26
+    float t = __saturatef(__fmaf_rn(q, M, 0.7992f * M)) + __saturatef(__fmaf_rn(q, M, 0.4824f * M));
+    t = t + __saturatef(__fmaf_rn(q, M, 0.2304f * M));
+    t = t + __saturatef(__fmul_rn(__saturatef(__fmul_rn(q, 0x1p100f)), 0x1p100f));
+    t = t + __saturatef(__fmaf_rn(q, M, -0.2304f * M));
+    t = t + __saturatef(__fmaf_rn(q, M, -0.4824f * M));
+    t = t + __saturatef(__fmaf_rn(q, M, -0.7992f * M));
+    return t;
+}
+
+// TQ3_CENTROIDS as printed on the page (fp32).
 __device__ __forceinline__ float centroid(uint32_t idx) {
     const uint32_t m = (idx & 4u) ? (idx & 3u) : (3u - idx);
     const float mag = m == 0 ? 0.1129f : m == 1 ? 0.3479f : m == 2 ? 0.6168f : 0.9816f;
     return (idx & 4u) ? mag : -mag;
 }
 
-// searchsorted(TQ3_BOUNDARIES, v, right=False): the number of boundaries strictly below v.
-__device__ __forceinline__ uint32_t bucketize(float v) {
-    return (uint32_t)(v > -0.7992f) + (uint32_t)(v > -0.4824f) + (uint32_t)(v > -0.2304f) +
-           (uint32_t)(v > 0.0f) + (uint32_t)(v > 0.2304f) + (uint32_t)(v > 0.4824f) +
-           (uint32_t)(v > 0.7992f);
+// Stages h = 2 .. 32 of the butterfly on 64 values held as 32 pairs (2k, 2k + 1).
+__device__ __forceinline__ void fwht_local_2_32(float (&a)[64]) {
+    f32x2 P[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) P[k] = pk2(a[2 * k], a[2 * k + 1]);
+#pragma unroll
+    for (int hp = 1; hp < 32; hp <<= 1)
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            if ((k & hp) == 0) {
+                const f32x2 A = P[k], B = P[k + hp];
+                P[k] = add2(A, B);
+                P[k + hp] = sub2(A, B);
+            }
+#pragma unroll
+    for (int k = 0; k < 32; ++k) upk2(P[k], a[2 * k], a[2 * k + 1]);
 }
 
-// fp32(1.0 / math.sqrt(128)), the post-multiplier of _fwht_inplace.
-__device__ __forceinline__ float fwht_post() { return __uint_as_float(0x3DB504F3u); }
-
-struct SignMask {
-    uint32_t w[4];  // bit i = sign draw i (1 -> +1, 0 -> -1)
-};
-
-// y * s_i for s_i = +-1 is exact: flip the sign bit where the draw was 0.
-__device__ __forceinline__ float apply_sign(float v, const SignMask &m, int i) {
-    const uint32_t keep = (m.w[i >> 5] >> (i & 31)) & 1u;
-    return __uint_as_float(__float_as_uint(v) ^ ((keep ^ 1u) << 31));
+__device__ __forceinline__ unsigned char *tile_base(unsigned char *raw) {
+    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
 }
 
-// _fwht_inplace without its final scaling: stages h = 1, 2, ..., 64 of (a, b) -> (a + b, a - b)
-// on positions (i, i + h) inside each 2h-block.
-__device__ __forceinline__ void fwht128(float (&a)[kD]) {
+// Address of 16-byte chunk j (0..7) of row `row` in a 128-byte-swizzled TMA box.
+__device__ __forceinline__ unsigned char *swz(unsigned char *box, int row, int j) {
+    return box + row * 128 + ((j ^ (row & 7)) << 4);
+}
+
+template <bool kBf16In, bool kDefault>
+__global__ void __launch_bounds__(kThreads, 4)
+    encode_kernel(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, SignMask mask,
+                  uint8_t *__restrict__ packed, float *__restrict__ norms, float *__restrict__ scales) {
+    constexpr int kBoxes = kBf16In ? 2 : 4;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *tile = tile_base(smem_raw);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(tile + kBoxes * kBoxBytes);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int half = lane >> 4;
+    const int row = warp * 16 + (lane & 15);
+    const int64_t v = (int64_t)blockIdx.x * kRows + row;
+
+    if (threadIdx.x == 0) mbar_init(bar, 1);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_expect_tx(bar, kBoxes * kBoxBytes);
 #pragma unroll
-    for (int h = 1; h < kD; h <<= 1) {
+        for (int b = 0; b < kBoxes; ++b)
+            tma_load_2d(tile + b * kBoxBytes, &tmap, b * (kBf16In ? 64 : 32), blockIdx.x * kRows, bar);
+    }
+    if (!mbar_wait_bounded(bar, 0, kMaxPolls)) {
+        if (lane == 0) atomicOr(&g_fault, 1u);
+        mbar_wait_bounded(bar, 0, kMaxPolls);  // give an in-flight copy a second chance to land
+        return;
+    }
+
+    const uint32_t H = half ? 0xffffffffu : 0u;
+    const uint32_t mlo = half ? mask.w[2] : mask.w[0], mhi = half ? mask.w[3] : mask.w[1];
+
+    // x.float() with the sign flips applied (exact), as 32 pairs (2k, 2k + 1)
+    float x[64];
+    if (kBf16In) {
+        unsigned char *box = tile + half * kBoxBytes;
 #pragma unroll
-        for (int i = 0; i < kD; ++i) {
-            if ((i & h) == 0) {
-                const float x = a[i], y = a[i + h];
-                a[i] = __fadd_rn(x, y);
-                a[i + h] = __fsub_rn(x, y);
+        for (int j = 0; j < 8; ++j) {
+            const uint4 q = *reinterpret_cast<const uint4 *>(swz(box, row, j));
+            const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int k = 4 * j + u;
+                const uint32_t w = w4[u] ^ pair_flip<kDefault>(k, H, mlo, mhi);
+                x[2 * k] = bf16_lo(w);
+                x[2 * k + 1] = bf16_hi(w);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            unsigned char *box = tile + (2 * half + (j >> 3)) * kBoxBytes;
+            const uint4 q = *reinterpret_cast<const uint4 *>(swz(box, row, j & 7));
+            const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int u = 0; u < 4; u += 2) {
+                const int k = 2 * j + u / 2;
+                const uint32_t f = pair_flip<kDefault>(k, H, mlo, mhi);
+                x[2 * k] = __uint_as_float(w4[u] ^ (f << 16));
+                x[2 * k + 1] = __uint_as_float(w4[u + 1] ^ (f & 0x80000000u));
             }
         }
     }
+
+    // Step 1: n = max(||x||, 1e-8); squares of fp32 values are exact in fp64
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const double d = (double)x[i];
+        acc[i & 3] = __fma_rn(d, d, acc[i & 3]);
+    }
+    const double mine = __dadd_rn(__dadd_rn(acc[0], acc[1]), __dadd_rn(acc[2], acc[3]));
+    const double other = __shfl_xor_sync(0xffffffffu, mine, 16);
+    const float n = fmaxf(__double2float_rn(__dsqrt_rn(__dadd_rn(mine, other))), 1e-8f);
+
+    // xn = x / n (signs already applied), then stage 1 of the FWHT
+    float a[64];
+    {
+        const float r = __frcp_rn(n);
+        const f32x2 R = pk2(r, r), ND = pk2(-n, -n);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) upk2(div2(pk2(x[2 * k], x[2 * k + 1]), R, ND), a[2 * k], a[2 * k + 1]);
+    }
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float p = a[2 * k], q = a[2 * k + 1];
+        a[2 * k] = __fadd_rn(p, q);
+        a[2 * k + 1] = __fsub_rn(p, q);
+    }
+    fwht_local_2_32(a);
+    // stage h = 64: element i (half 0) with element i + 64 (half 1)
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, a[i], 16);
+        a[i] = half ? __fsub_rn(o, a[i]) : __fadd_rn(a[i], o);
+    }
+
+    // Step 4: scale = max(max|xh|, 1e-8) with xh = fwht * c; max|fl(y c)| = fl(max|y| c)
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 64; i += 2) m = max3(m, fabsf(a[i]), fabsf(a[i + 1]));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+    const float c = fwht_post();
+    const float s = fmaxf(__fmul_rn(m, c), 1e-8f);
+
+    // Steps 5-6: idx = bucketize(RN(RN(y c) / s)), 8 indices per 24-bit little-endian group
+    uint32_t grp[8];
+    {
+        const float rs = __frcp_rn(s);
+        const f32x2 C2 = pk2(c, c), RS = pk2(rs, rs), NS = pk2(-s, -s);
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            float wf = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+                float q0, q1;
+                upk2(div2(mul2(pk2(a[8 * g + i], a[8 * g + i + 1]), C2), RS, NS), q0, q1);
+                wf = __fmaf_rn(bucket_steps(q0), (float)(1u << (3 * i)), wf);
+                wf = __fmaf_rn(bucket_steps(q1), (float)(1u << (3 * i + 3)), wf);
+            }
+            grp[g] = __float2uint_rz(wf);  // exact: an integer below 2^24
+        }
+    }
+    if (v < n_vec) {
+        // this thread's 24 bytes are 48v + 24 * half ...; both halves write one 16-byte chunk at
+        // 48v + 32 * half and one 8-byte chunk at 48v + 16 + 8 * half (aligned for either half,
+        // with no lane-divergent branch around the accesses)
+        const uint32_t w0 = grp[0] | (grp[1] << 24), w1 = (grp[1] >> 8) | (grp[2] << 16),
+                       w2 = (grp[2] >> 16) | (grp[3] << 8);
+        const uint32_t w3 = grp[4] | (grp[5] << 24), w4 = (grp[5] >> 8) | (grp[6] << 16),
+                       w5 = (grp[6] >> 16) | (grp[7] << 8);
+        uint8_t *rec = packed + v * 48;
+        st_stream16(rec + 32 * half, half ? make_uint4(w2, w3, w4, w5) : make_uint4(w0, w1, w2, w3));
+        st_stream8(rec + 16 + 8 * half, half ? make_uint2(w0, w1) : make_uint2(w4, w5));
+        if (half == 0)
+            norms[v] = n;
+        else
+            scales[v] = s;
+    }
 }
 
-template <bool kBf16In>
-__global__ void __launch_bounds__(kThreads)
-    encode_kernel(const void *__restrict__ xin, int64_t n_vec, SignMask mask,
-                  uint8_t *__restrict__ packed, float *__restrict__ norms,
-                  float *__restrict__ scales) {
-    const int64_t v = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (v >= n_vec) return;
-
-    // x.float(): bf16 widening is exact.
-    float a[kD];
-    if (kBf16In) {
-        const uint8_t *src = static_cast<const uint8_t *>(xin) + v * (kD * 2);
-#pragma unroll
-        for (int q = 0; q < kD / 8; ++q) {
-            const uint4 u = ld_stream16(src + 16 * q);
-            a[8 * q + 0] = bf16_lo(u.x);
-            a[8 * q + 1] = bf16_hi(u.x);
-            a[8 * q + 2] = bf16_lo(u.y);
-            a[8 * q + 3] = bf16_hi(u.y);
-            a[8 * q + 4] = bf16_lo(u.z);
-            a[8 * q + 5] = bf16_hi(u.z);
-            a[8 * q + 6] = bf16_lo(u.w);
-            a[8 * q + 7] = bf16_hi(u.w);
-        }
-    } else {
-        const uint8_t *src = static_cast<const uint8_t *>(xin) + v * (kD * 4);
-#pragma unroll
-        for (int q = 0; q < kD / 4; ++q) {
-            const uint4 u = ld_stream16(src + 16 * q);
-            a[4 * q + 0] = __uint_as_float(u.x);
-            a[4 * q + 1] = __uint_as_float(u.y);
-            a[4 * q + 2] = __uint_as_float(u.z);
-            a[4 * q + 3] = __uint_as_float(u.w);
-        }
-    }
-
-    // Step 1: n = max(||x||, 1e-8). Squares of fp32 values are exact in fp64.
-    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-#pragma unroll
-    for (int i = 0; i < kD; i += 4) {
-        s0 = __dadd_rn(s0, __dmul_rn((double)a[i + 0], (double)a[i + 0]));
-        s1 = __dadd_rn(s1, __dmul_rn((double)a[i + 1], (double)a[i + 1]));
-        s2 = __dadd_rn(s2, __dmul_rn((double)a[i + 2], (double)a[i + 2]));
-        s3 = __dadd_rn(s3, __dmul_rn((double)a[i + 3], (double)a[i + 3]));
-    }
-    float n = __double2float_rn(__dsqrt_rn(__dadd_rn(__dadd_rn(s0, s1), __dadd_rn(s2, s3))));
-    n = fmaxf(n, 1e-8f);
-
-    // xn = x / n, then the sign flips (exact), then the FWHT and its fp32 post-multiplier.
-#pragma unroll
-    for (int i = 0; i < kD; ++i) a[i] = apply_sign(__fdiv_rn(a[i], n), mask, i);
-    fwht128(a);
-    const float post = fwht_post();
-#pragma unroll
-    for (int i = 0; i < kD; ++i) a[i] = __fmul_rn(a[i], post);
-
-    // Step 4: absmax scale, clamp(min=1e-8).
-    float s = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kD; ++i) s = fmaxf(s, fabsf(a[i]));
-    s = fmaxf(s, 1e-8f);
-
-    // Steps 5-6: indices of xs = xh / s, packed 8 per 24-bit little-endian group.
-    uint32_t grp[16];
-#pragma unroll
-    for (int g = 0; g < 16; ++g) {
-        uint32_t bits = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) bits |= bucketize(__fdiv_rn(a[8 * g + i], s)) << (3 * i);
-        grp[g] = bits;
-    }
-    uint8_t *dst = packed + v * 48;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        // groups 4c..4c+3 are 96 bits = three 32-bit little-endian words
-        const uint32_t g0 = grp[4 * c], g1 = grp[4 * c + 1], g2 = grp[4 * c + 2], g3 = grp[4 * c + 3];
-        grp[4 * c + 0] = g0 | (g1 << 24);
-        grp[4 * c + 1] = (g1 >> 8) | (g2 << 16);
-        grp[4 * c + 2] = (g2 >> 16) | (g3 << 8);
-    }
-    st_stream16(dst + 0, make_uint4(grp[0], grp[1], grp[2], grp[4]));
-    st_stream16(dst + 16, make_uint4(grp[5], grp[6], grp[8], grp[9]));
-    st_stream16(dst + 32, make_uint4(grp[10], grp[12], grp[13], grp[14]));
-    norms[v] = n;
-    scales[v] = s;
-}
-
-template <bool kBf16Out>
-__global__ void __launch_bounds__(kThreads)
+template <bool kBf16Out, bool kDefault>
+__global__ void __launch_bounds__(kThreads, 4)
     decode_kernel(const uint8_t *__restrict__ packed, const float *__restrict__ norms,
-                  const float *__restrict__ scales, int64_t n_vec, SignMask mask,
-                  void *__restrict__ out) {
-    const int64_t v = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (v >= n_vec) return;
+                  const float *__restrict__ scales, int64_t n_vec, SignMask mask, void *__restrict__ out) {
+    constexpr int kBoxes = kBf16Out ? 2 : 4;
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ float ctab[8];
+    unsigned char *tile = tile_base(smem_raw);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int half = lane >> 4;
+    const int row = warp * 16 + (lane & 15);
+    const int64_t v = (int64_t)blockIdx.x * kRows + row;
+    if (threadIdx.x < 8) ctab[threadIdx.x] = centroid(threadIdx.x);
 
-    const uint8_t *src = packed + v * 48;
-    const uint4 p0 = ld_stream16(src), p1 = ld_stream16(src + 16), p2 = ld_stream16(src + 32);
-    const uint32_t w[12] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w, p2.x, p2.y, p2.z, p2.w};
-    const float scale = scales[v];
-    const float n = norms[v];
+    // this thread's 64 indices: bytes 24 * half .. 24 * half + 23 of the 48-byte record
+    uint32_t pw[6] = {0, 0, 0, 0, 0, 0};
+    float n = 0.0f, scale = 0.0f;
+    if (v < n_vec) {
+        // bytes 48v + 24 * half ... as one 16-byte chunk at 48v + 32 * half and one 8-byte chunk at
+        // 48v + 16 + 8 * half: aligned for either half, no lane-divergent branch around the loads
+        const uint8_t *rec = packed + v * 48;
+        const uint4 c16 = ld_stream16(rec + 32 * half);
+        const uint2 c8 = ld_stream8(rec + 16 + 8 * half);
+        pw[0] = half ? c8.x : c16.x;
+        pw[1] = half ? c8.y : c16.y;
+        pw[2] = half ? c16.x : c16.z;
+        pw[3] = half ? c16.y : c16.w;
+        pw[4] = half ? c16.z : c8.x;
+        pw[5] = half ? c16.w : c8.y;
+        n = norms[v];
+        scale = scales[v];
+    }
+    __syncthreads();  // ctab
 
-    // _unpack_3bit, centroids[idx] * scale
-    float a[kD];
+    // _unpack_3bit, then centroids[idx] * scale
+    float a[64];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const uint32_t w0 = w[3 * c], w1 = w[3 * c + 1], w2 = w[3 * c + 2];
-        const uint32_t g[4] = {w0 & 0xffffffu, (w0 >> 24) | ((w1 & 0xffffu) << 8),
-                               (w1 >> 16) | ((w2 & 0xffu) << 16), w2 >> 8};
+    for (int c2 = 0; c2 < 2; ++c2) {
+        const uint32_t w0 = pw[3 * c2], w1 = pw[3 * c2 + 1], w2 = pw[3 * c2 + 2];
+        const uint32_t g[4] = {w0 & 0xffffffu, (w0 >> 24) | ((w1 & 0xffffu) << 8), (w1 >> 16) | ((w2 & 0xffu) << 16),
+                               w2 >> 8};
 #pragma unroll
         for (int k = 0; k < 4; ++k)
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                a[32 * c + 8 * k + i] = __fmul_rn(centroid((g[k] >> (3 * i)) & 7u), scale);
+            for (int i = 0; i < 8; ++i) a[32 * c2 + 8 * k + i] = __fmul_rn(ctab[(g[k] >> (3 * i)) & 7u], scale);
     }
-
-    // inverse FWHT (the normalised transform is its own inverse), then signs, then the norm
-    fwht128(a);
-    const float post = fwht_post();
+    // the normalised FWHT (its own inverse)
 #pragma unroll
-    for (int i = 0; i < kD; ++i) a[i] = __fmul_rn(apply_sign(__fmul_rn(a[i], post), mask, i), n);
-
+    for (int k = 0; k < 32; ++k) {
+        const float p = a[2 * k], q = a[2 * k + 1];
+        a[2 * k] = __fadd_rn(p, q);
+        a[2 * k + 1] = __fsub_rn(p, q);
+    }
+    fwht_local_2_32(a);
+#pragma unroll
+    for (int i = 0; i < 64; ++i) {
+        const float o = __shfl_xor_sync(0xffffffffu, a[i], 16);
+        a[i] = half ? __fsub_rn(o, a[i]) : __fadd_rn(a[i], o);
+    }
+    // * post, then * norm; the sign flips (exact) are applied to the output bits
+    {
+        const float post = fwht_post();
+        const f32x2 P2 = pk2(post, post), N2 = pk2(n, n);
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            upk2(mul2(mul2(pk2(a[2 * k], a[2 * k + 1]), P2), N2), a[2 * k], a[2 * k + 1]);
+    }
+    const uint32_t H = half ? 0xffffffffu : 0u;
+    const uint32_t mlo = half ? mask.w[2] : mask.w[0], mhi = half ? mask.w[3] : mask.w[1];
     if (kBf16Out) {
-        uint8_t *dst = static_cast<uint8_t *>(out) + v * (kD * 2);
+        unsigned char *box = tile + half * kBoxBytes;
 #pragma unroll
-        for (int q = 0; q < kD / 8; ++q)
-            st_stream16(dst + 16 * q,
-                        make_uint4(pack_bf16x2(a[8 * q + 0], a[8 * q + 1]), pack_bf16x2(a[8 * q + 2], a[8 * q + 3]),
-                                   pack_bf16x2(a[8 * q + 4], a[8 * q + 5]), pack_bf16x2(a[8 * q + 6], a[8 * q + 7])));
+        for (int j = 0; j < 8; ++j) {
+            uint32_t o[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int k = 4 * j + u;
+                o[u] = pack_bf16x2(a[2 * k], a[2 * k + 1]) ^ pair_flip<kDefault>(k, H, mlo, mhi);
+            }
+            *reinterpret_cast<uint4 *>(swz(box, row, j)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     } else {
-        uint8_t *dst = static_cast<uint8_t *>(out) + v * (kD * 4);
 #pragma unroll
-        for (int q = 0; q < kD / 4; ++q)
-            st_stream16(dst + 16 * q, make_uint4(__float_as_uint(a[4 * q + 0]), __float_as_uint(a[4 * q + 1]),
-                                                 __float_as_uint(a[4 * q + 2]), __float_as_uint(a[4 * q + 3])));
+        for (int j = 0; j < 16; ++j) {
+            unsigned char *box = tile + (2 * half + (j >> 3)) * kBoxBytes;
+            uint32_t o[4];
+#pragma unroll
+            for (int u = 0; u < 4; u += 2) {
+                const int k = 2 * j + u / 2;
+                const uint32_t f = pair_flip<kDefault>(k, H, mlo, mhi);
+                o[u] = __float_as_uint(a[2 * k]) ^ (f << 16);
+                o[u + 1] = __float_as_uint(a[2 * k + 1]) ^ (f & 0x80000000u);
+            }
+            *reinterpret_cast<uint4 *>(swz(box, row, j & 7)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
+    __syncthreads();
+    // write the tile back with coalesced 16-byte stores: the CTA's rows are one contiguous range
+    constexpr int kChunksPerRow = kBoxes * 8;
+    const int64_t rows_left = n_vec - (int64_t)blockIdx.x * kRows;
+    unsigned char *gdst = static_cast<unsigned char *>(out) + (int64_t)blockIdx.x * kRows * (kChunksPerRow * 16);
+#pragma unroll
+    for (int it = 0; it < kChunksPerRow * kRows / kThreads; ++it) {
+        const int chunk = it * kThreads + threadIdx.x;
+        const int r = chunk / kChunksPerRow, cj = chunk % kChunksPerRow;
+        if (r < rows_left) {
+            const uint4 val = *reinterpret_cast<const uint4 *>(swz(tile + (cj >> 3) * kBoxBytes, r, cj & 7));
+            st_stream16(gdst + (int64_t)chunk * 16, val);
+        }
     }
 }
 
-inline unsigned grid_for(int64_t n_vec) { return (unsigned)((n_vec + kThreads - 1) / kThreads); }
+inline bool is_default(const SignMask &m) {
+    for (int i = 0; i < 4; ++i)
+        if (m.w[i] != default_mask_word(i)) return false;
+    return true;
+}
+
+inline size_t smem_bytes(bool bf16) { return (size_t)(bf16 ? 2 : 4) * kBoxBytes + 1024 + 64; }
 
 }  // namespace tq3
 }  // namespace wq
@@ -219,12 +398,32 @@ extern "C" wq_status tq3_encode(const void *x, int x_dtype, int64_t n_vec, const
     if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(norms, 4) || !aligned(scales, 4)) return WQ_ERR_ALIGN;
     tq3::SignMask m;
     for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
+    const bool def = tq3::is_default(m), bf = x_dtype == WQ_BF16;
+    const int esz = bf ? 2 : 4;
+    const size_t smem = tq3::smem_bytes(bf);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (x_dtype == WQ_BF16)
-        tq3::encode_kernel<true><<<tq3::grid_for(n_vec), tq3::kThreads, 0, s>>>(x, n_vec, m, packed, norms, scales);
-    else
-        tq3::encode_kernel<false><<<tq3::grid_for(n_vec), tq3::kThreads, 0, s>>>(x, n_vec, m, packed, norms, scales);
-    return launch_status();
+    for (int64_t off = 0; off < n_vec; off += tq3::kMaxChunk) {
+        const int64_t cnt = n_vec - off < tq3::kMaxChunk ? n_vec - off : tq3::kMaxChunk;
+        const unsigned char *xc = static_cast<const unsigned char *>(x) + off * (tq3::kD * esz);
+        CUtensorMap tm;
+        if (!make_tmap_2d(&tm, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, xc, tq3::kD,
+                          (uint64_t)cnt, tq3::kD * esz, bf ? 64 : 32, tq3::kRows))
+            return WQ_ERR_CUDA;
+        const unsigned grid = (unsigned)((cnt + tq3::kRows - 1) / tq3::kRows);
+        uint8_t *pc = packed + off * 48;
+        float *nc = norms + off, *sc = scales + off;
+        if (bf && def)
+            tq3::encode_kernel<true, true><<<grid, tq3::kThreads, smem, s>>>(cnt, tm, m, pc, nc, sc);
+        else if (bf)
+            tq3::encode_kernel<true, false><<<grid, tq3::kThreads, smem, s>>>(cnt, tm, m, pc, nc, sc);
+        else if (def)
+            tq3::encode_kernel<false, true><<<grid, tq3::kThreads, smem, s>>>(cnt, tm, m, pc, nc, sc);
+        else
+            tq3::encode_kernel<false, false><<<grid, tq3::kThreads, smem, s>>>(cnt, tm, m, pc, nc, sc);
+        const wq_status st = launch_status();
+        if (st != WQ_OK) return st;
+    }
+    return WQ_OK;
 }
 
 extern "C" wq_status tq3_decode(const uint8_t *packed, const float *norms, const float *scales, int64_t n_vec,
@@ -237,15 +436,40 @@ extern "C" wq_status tq3_decode(const uint8_t *packed, const float *norms, const
     if (!aligned(packed, 16) || !aligned(out, 16) || !aligned(norms, 4) || !aligned(scales, 4)) return WQ_ERR_ALIGN;
     tq3::SignMask m;
     for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
+    const bool def = tq3::is_default(m), bf = out_dtype == WQ_BF16;
+    const int esz = bf ? 2 : 4;
+    const size_t smem = tq3::smem_bytes(bf);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (out_dtype == WQ_BF16)
-        tq3::decode_kernel<true><<<tq3::grid_for(n_vec), tq3::kThreads, 0, s>>>(packed, norms, scales, n_vec, m, out);
-    else
-        tq3::decode_kernel<false><<<tq3::grid_for(n_vec), tq3::kThreads, 0, s>>>(packed, norms, scales, n_vec, m, out);
-    return launch_status();
+    for (int64_t off = 0; off < n_vec; off += tq3::kMaxChunk) {
+        const int64_t cnt = n_vec - off < tq3::kMaxChunk ? n_vec - off : tq3::kMaxChunk;
+        unsigned char *oc = static_cast<unsigned char *>(out) + off * (tq3::kD * esz);
+        const unsigned grid = (unsigned)((cnt + tq3::kRows - 1) / tq3::kRows);
+        const uint8_t *pc = packed + off * 48;
+        const float *nc = norms + off, *sc = scales + off;
+        if (bf && def)
+            tq3::decode_kernel<true, true><<<grid, tq3::kThreads, smem, s>>>(pc, nc, sc, cnt, m, oc);
+        else if (bf)
+            tq3::decode_kernel<true, false><<<grid, tq3::kThreads, smem, s>>>(pc, nc, sc, cnt, m, oc);
+        else if (def)
+            tq3::decode_kernel<false, true><<<grid, tq3::kThreads, smem, s>>>(pc, nc, sc, cnt, m, oc);
+        else
+            tq3::decode_kernel<false, false><<<grid, tq3::kThreads, smem, s>>>(pc, nc, sc, cnt, m, oc);
+        const wq_status st = launch_status();
+        if (st != WQ_OK) return st;
+    }
+    return WQ_OK;
 }
 
 extern "C" int64_t tq3_compressed_bytes(int64_t n_vec) {
     if (n_vec < 0 || n_vec > INT64_MAX / 56) return -1;
     return n_vec * 56;
+}
+
+extern "C" wq_status wq_device_fault(unsigned int *flags) {
+    if (!flags) return WQ_ERR_NULL;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, tq3::g_fault, sizeof v) != cudaSuccess) return WQ_ERR_CUDA;
+    if (v && cudaMemcpyToSymbol(tq3::g_fault, &zero, sizeof zero) != cudaSuccess) return WQ_ERR_CUDA;
+    *flags = v;
+    return WQ_OK;
 }

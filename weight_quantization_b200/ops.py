@@ -31,6 +31,7 @@ PROTOTYPES = {
     "rpbh_packed_bytes": (_i64, [_i64, _i64, _int]),
     "wq_gaussian_lloyd_max": (_int, [_int, _int, _vp]),
     "wq_rpbh_codebook": (_int, [_int, _i64, _vp]),
+    "wq_device_fault": (_int, [_vp]),
     "wq_status_string": (C.c_char_p, [_int]),
     "wq_version": (_int, []),
 }
@@ -199,6 +200,13 @@ def gaussian_lloyd_max(bits: int, iters: int = 200) -> np.ndarray:
     out = np.zeros(1 << bits, np.float32)
     _check("wq_gaussian_lloyd_max", lib().wq_gaussian_lloyd_max(bits, iters, out.ctypes.data))
     return out
+
+
+def device_fault() -> int:
+    """Read and clear the sticky fault bits (non-zero if a kernel's bounded TMA wait ran out)."""
+    v = C.c_uint(0)
+    _check("wq_device_fault", lib().wq_device_fault(C.byref(v)))
+    return int(v.value)
 
 
 def rpbh_codebook(bits: int, d: int) -> np.ndarray:
