@@ -50,7 +50,8 @@ def _quantize_and_check(wq, oracle, w, is_bf16, d, bits):
     return st, packed, norms
 
 
-@pytest.mark.parametrize("d,rows", [(32, 5), (96, 37), (256, 3), (1024, 9), (3072, 17), (640, 1)])
+@pytest.mark.parametrize("d,rows", [(32, 5), (96, 37), (192, 11), (256, 3), (1024, 9), (3072, 17), (640, 1),
+                                    (4096, 3), (12288, 2)])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 @pytest.mark.parametrize("is_bf16", [False, True])
 def test_quantize_small(wq, oracle, d, rows, bits, is_bf16):
@@ -88,7 +89,8 @@ def test_quantize_dit_weights_full_size(wq, oracle, rows):
     print("rpbh quantize C5", rows, st)
 
 
-@pytest.mark.parametrize("d,rows,bits", [(96, 7, 2), (1024, 5, 3), (3072, 33, 4), (11008, 4, 3)])
+@pytest.mark.parametrize("d,rows,bits", [(96, 7, 2), (192, 3, 3), (1024, 5, 3), (3072, 33, 4), (11008, 4, 3),
+                                         (4096, 2, 2)])
 @pytest.mark.parametrize("norm_bf16", [False, True])
 @pytest.mark.parametrize("out_bf16", [False, True])
 @pytest.mark.parametrize("unrotate", [False, True])
@@ -136,7 +138,8 @@ def test_quantize_then_dequantize_llm_roundtrip(wq, oracle):
     assert cos.mean().item() > 0.96
 
 
-@pytest.mark.parametrize("rows,d", [(2048, 11008), (4096, 3072), (3, 96), (1, 32)])
+@pytest.mark.parametrize("rows,d", [(2048, 11008), (4096, 3072), (3, 96), (1, 32), (5, 192), (3, 4096),
+                                    (7, 640)])
 def test_rotate_activations(wq, oracle, rows, d):
     perm, signs, perm_d, signs_d = _params(d)
     h = d & -d
@@ -170,3 +173,28 @@ def test_rpbh_errors(wq):
     with pytest.raises(wq.WQError) as e:
         wq.rpbh_rotate_activations(torch.zeros(4, 100, device="cuda"), perm_d, signs_d)
     assert e.value.status == -6
+
+
+def test_asymmetric_codebook_takes_generic_bucketize(wq, oracle):
+    """A caller-supplied codebook that is not antisymmetric is bucketized edge by edge."""
+    d, rows, bits = 3072, 6, 3
+    perm, signs, perm_d, signs_d = _params(d)
+    cb = (oracle.rpbh_codebook(bits, d) + np.float32(0.001)).astype(np.float32)
+    w = inputs.gaussian((rows, d), seed=91) * 0.02
+    packed, norms = wq.rpbh_quantize_weight(_t(w), perm_d, signs_d, bits, cb)
+    st, _, ref_norms = parity.check_rpbh_quantize(oracle, w, False, perm, signs, d & -d, cb, bits, packed.cpu().numpy())
+    assert st["bytes_equal"]
+    parity.check_norms(norms.cpu().numpy(), ref_norms)
+
+
+def test_misaligned_tables_take_generic_path(wq, oracle):
+    """perm/signs that are only 4-byte aligned still work (the general kernels take them)."""
+    d, rows = 1024, 4
+    perm, signs = inputs.rpbh_params(d)
+    pbuf = torch.zeros(d + 1, dtype=torch.int32, device="cuda")
+    pbuf[1:] = torch.from_numpy(perm).cuda()
+    sbuf = torch.zeros(d + 1, dtype=torch.int8, device="cuda")
+    sbuf[1:] = torch.from_numpy(signs).cuda()
+    x = inputs.activations(rows, d, seed=92)
+    out = wq.rpbh_rotate_activations(_t(x, True), pbuf[1:], sbuf[1:])
+    assert np.array_equal(_np16(out), oracle.rpbh_rotate_bf16(x, perm, signs, d & -d))

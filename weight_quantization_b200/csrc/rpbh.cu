@@ -11,6 +11,7 @@
 #include <cmath>
 
 #include "common.cuh"
+#include "rpbh_fast.cuh"
 #include "wq.h"
 
 namespace wq {
@@ -254,9 +255,11 @@ extern "C" wq_status rpbh_rotate_activations(const void *x, int dtype, int64_t r
     if (rows == 0) return WQ_OK;
     if (!x || !perm || !signs || !x_rot) return WQ_ERR_NULL;
     if (!aligned(x, 16) || !aligned(x_rot, 16) || !aligned(perm, 4)) return WQ_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (rpbh_fast::supported(d, dtype_size(dtype), dtype_size(dtype)) && aligned(perm, 16) && aligned(signs, 16))
+        return rpbh_fast::rotate(x, dtype, rows, d, perm, signs, x_rot, s);
     const int h = (int)(d & -d);
     const size_t smem = (size_t)d * (4 + dtype_size(dtype));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     const float post = rpbh::fwht_post(h);
     if (dtype == WQ_BF16) {
         if ((st = rpbh::prepare(rpbh::rotate_kernel<true>, smem)) != WQ_OK) return st;
@@ -279,11 +282,13 @@ extern "C" wq_status rpbh_quantize_weight(const void *W, int w_dtype, int64_t ro
     if (!W || !perm || !signs || !codebook || !packed || !row_norms) return WQ_ERR_NULL;
     if (!aligned(W, 16) || !aligned(packed, 4) || !aligned(perm, 4) || !aligned(row_norms, dtype_size(w_dtype)))
         return WQ_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (rpbh_fast::supported(d, dtype_size(w_dtype), 1) && aligned(perm, 16) && aligned(signs, 16))
+        return rpbh_fast::quantize(W, w_dtype, rows, d, perm, signs, bits, codebook, packed, row_norms, s);
     rpbh::Codebook cb = {};
     for (int k = 0; k < (1 << bits); ++k) cb.c[k] = codebook[k];
     const int h = (int)(d & -d);
     const size_t smem = (size_t)d * (4 + dtype_size(w_dtype));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     const float post = rpbh::fwht_post(h);
     if (w_dtype == WQ_BF16) {
         if ((st = rpbh::prepare(rpbh::quantize_kernel<true>, smem)) != WQ_OK) return st;
@@ -327,9 +332,12 @@ extern "C" wq_status rpbh_dequantize_weight(const uint8_t *packed, const void *r
     if (!aligned(packed, 4) || !aligned(out, 16) || !aligned(row_norms, dtype_size(norm_dtype)) ||
         (unrotate && !aligned(perm, 4)))
         return WQ_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (unrotate && rpbh_fast::supported(d, 1, dtype_size(out_dtype)) && aligned(perm, 16) && aligned(signs, 16))
+        return rpbh_fast::dequantize_unrotate(packed, row_norms, norm_dtype, rows, d, bits, codebook, perm, signs, out,
+                                              out_dtype, s);
     rpbh::Codebook cb = {};
     for (int k = 0; k < (1 << bits); ++k) cb.c[k] = codebook[k];
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int di = (int)d;
     const bool nb = norm_dtype == WQ_BF16, ob = out_dtype == WQ_BF16;
 #define WQ_DQ(NB, OB, UR) launch_dequant<NB, OB, UR>(packed, row_norms, rows, di, bits, cb, perm, signs, out, s)

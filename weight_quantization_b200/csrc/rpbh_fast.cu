@@ -1,0 +1,556 @@
+// Register-blocked RPBH kernels on sm_100a: page "orbit_quant.py" (rpbh_forward, _fwht,
+// _quantize_rows, pack_codes, unpack_codes, dequantize / rpbh_inverse).
+//
+// For a Hadamard block h = 2^(2B) each h-block is viewed as an S x S matrix (S = 2^B, element
+// k = row * S + col). Butterfly stages 1 .. S/2 act on the column index and stages S .. h/2 on
+// the row index, so the block FWHT is two passes of in-register butterflies over S values:
+//   pass 0: one thread takes one matrix row (S contiguous elements), gathers them through the
+//           permutation from the row staged in shared memory, applies the signs and the first B
+//           stages, and writes the row to a transpose buffer;
+//   pass 1: one thread takes one matrix column, applies the remaining B stages and the epilogue.
+// Stages stay in the page's order (h = 1, 2, 4, ...) and every butterfly is one IEEE add or
+// subtract, so results match the stage-by-stage definition bit for bit. The transpose buffer
+// swizzles 16-byte chunks by row (and flips the row parity of odd blocks when S < 32) so that
+// pass 0's 16-byte stores and pass 1's 4-byte loads are free of shared-memory bank conflicts.
+// One CTA owns one weight/activation row; the row norm of the quantizer is a CTA reduction.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cmath>
+
+#include "common.cuh"
+#include "rpbh_fast.cuh"
+
+namespace wq {
+namespace rpbh_fast {
+
+constexpr int kMaxThreads = 256;
+
+template <int B>
+struct Geo {
+    static constexpr int S = 1 << B;
+    static constexpr int H = 1 << (2 * B);
+    static constexpr int NCH = S / 4;
+    static constexpr bool kParity = S < 32;
+};
+
+template <int B>
+__device__ __forceinline__ int chunk_swz(int row) {
+    return B == 3 ? ((row >> 2) & 1) : B == 4 ? ((row >> 1) & 3) : (row & 7);
+}
+
+// Physical float index of element (row, col) of h-block `blk` in the transpose buffer.
+template <int B>
+__device__ __forceinline__ int bufpos(int blk, int row, int col) {
+    using G = Geo<B>;
+    const int prow = G::kParity ? (row ^ (blk & 1)) : row;
+    const int ch = (col >> 2) ^ (chunk_swz<B>(row) & (G::NCH - 1));
+    return blk * G::H + prow * G::S + ch * 4 + (col & 3);
+}
+
+// Stages 1, 2, ..., S/2 of the butterfly on S register values; pairs are packed two at a time
+// from the second stage on.
+template <int S>
+__device__ __forceinline__ void butterfly(float (&y)[S]) {
+#pragma unroll
+    for (int k = 0; k < S; k += 2) {
+        const float p = y[k], q = y[k + 1];
+        y[k] = __fadd_rn(p, q);
+        y[k + 1] = __fsub_rn(p, q);
+    }
+    f32x2 P[S / 2];
+#pragma unroll
+    for (int k = 0; k < S / 2; ++k) P[k] = pk2(y[2 * k], y[2 * k + 1]);
+#pragma unroll
+    for (int hp = 1; hp < S / 2; hp <<= 1)
+#pragma unroll
+        for (int k = 0; k < S / 2; ++k)
+            if ((k & hp) == 0) {
+                const f32x2 A = P[k], Bv = P[k + hp];
+                P[k] = add2(A, Bv);
+                P[k + hp] = sub2(A, Bv);
+            }
+#pragma unroll
+    for (int k = 0; k < S / 2; ++k) upk2(P[k], y[2 * k], y[2 * k + 1]);
+}
+
+__device__ __forceinline__ unsigned char *align16(unsigned char *p) {
+    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 15) & ~uintptr_t(15));
+}
+
+// Copy `bytes` (a multiple of 16) global -> shared with 16-byte accesses.
+__device__ __forceinline__ void copy_in(unsigned char *dst, const unsigned char *src, int bytes) {
+    for (int c = threadIdx.x; c < bytes / 16; c += blockDim.x)
+        *reinterpret_cast<uint4 *>(dst + 16 * c) = ld_stream16(src + 16 * (size_t)c);
+}
+__device__ __forceinline__ void copy_out(unsigned char *dst, const unsigned char *src, int bytes) {
+    for (int c = threadIdx.x; c < bytes / 16; c += blockDim.x)
+        st_stream16(dst + 16 * (size_t)c, *reinterpret_cast<const uint4 *>(src + 16 * c));
+}
+
+__device__ __forceinline__ int clampi(int32_t p, int d) { return (uint32_t)p < (uint32_t)d ? p : 0; }
+
+// pass 0 for one matrix row: y[t] = x[perm[j0 + t]] * signs[j0 + t], then the first B stages
+template <int B, bool kBf16>
+__device__ __forceinline__ void gather_row(float (&y)[1 << B], const unsigned char *raw, int j0, int d,
+                                           const int32_t *__restrict__ perm, const int8_t *__restrict__ signs) {
+    constexpr int S = 1 << B;
+    int32_t pi[S];
+#pragma unroll
+    for (int q = 0; q < S / 4; ++q) {
+        const int4 v = __ldg(reinterpret_cast<const int4 *>(perm + j0) + q);
+        pi[4 * q] = v.x; pi[4 * q + 1] = v.y; pi[4 * q + 2] = v.z; pi[4 * q + 3] = v.w;
+    }
+    uint32_t sw[S / 4];
+    if (S >= 16) {
+#pragma unroll
+        for (int q = 0; q < S / 16; ++q) {
+            const int4 v = __ldg(reinterpret_cast<const int4 *>(signs + j0) + q);
+            sw[4 * q] = v.x; sw[4 * q + 1] = v.y; sw[4 * q + 2] = v.z; sw[4 * q + 3] = v.w;
+        }
+    } else {
+        const int2 v = __ldg(reinterpret_cast<const int2 *>(signs + j0));
+        sw[0] = v.x; sw[1] = v.y;
+    }
+#pragma unroll
+    for (int t = 0; t < S; ++t) {
+        const int p = clampi(pi[t], d);
+        const float xv = kBf16 ? bf16_to_f32(reinterpret_cast<const uint16_t *>(raw)[p])
+                               : reinterpret_cast<const float *>(raw)[p];
+        const float sg = (float)(int8_t)(sw[t >> 2] >> (8 * (t & 3)));
+        y[t] = __fmul_rn(xv, sg);  // index_select(x, perm) * signs (exact)
+    }
+    butterfly<S>(y);
+}
+
+template <int B>
+__device__ __forceinline__ void store_row(unsigned char *buf_raw, const float (&y)[1 << B], int blk, int r) {
+    constexpr int S = 1 << B;
+    float *buf = reinterpret_cast<float *>(buf_raw);
+#pragma unroll
+    for (int q = 0; q < S / 4; ++q)
+        *reinterpret_cast<float4 *>(buf + bufpos<B>(blk, r, 4 * q)) =
+            make_float4(y[4 * q], y[4 * q + 1], y[4 * q + 2], y[4 * q + 3]);
+}
+
+template <int B>
+__device__ __forceinline__ void load_col(float (&y)[1 << B], const unsigned char *buf_raw, int blk, int c) {
+    constexpr int S = 1 << B;
+    const float *buf = reinterpret_cast<const float *>(buf_raw);
+#pragma unroll
+    for (int t = 0; t < S; ++t) y[t] = buf[bufpos<B>(blk, t, c)];
+}
+
+// ---------------------------------------------------------------------------------------------
+// rpbh_rotate_activations: x_rot = blkdiag(H_h) D P x, computed in fp32, rounded once.
+// ---------------------------------------------------------------------------------------------
+template <int B, bool kBf16>
+__global__ void __launch_bounds__(kMaxThreads)
+    rotate_kernel(const void *__restrict__ x, int d, float post, const int32_t *__restrict__ perm,
+                  const int8_t *__restrict__ signs, void *__restrict__ out) {
+    using G = Geo<B>;
+    constexpr int esz = kBf16 ? 2 : 4;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *raw = align16(smem_raw);
+    unsigned char *buf = raw + (size_t)d * esz;
+    const int64_t row = blockIdx.x;
+    copy_in(raw, static_cast<const unsigned char *>(x) + row * (int64_t)d * esz, d * esz);
+    __syncthreads();
+    const int nslots = d >> B;
+    for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+        const int blk = s >> B, r = s & (G::S - 1);
+        float y[G::S];
+        gather_row<B, kBf16>(y, raw, blk * G::H + r * G::S, d, perm, signs);
+        store_row<B>(buf, y, blk, r);
+    }
+    __syncthreads();
+    for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+        const int blk = s >> B, c = s & (G::S - 1);
+        float y[G::S];
+        load_col<B>(y, buf, blk, c);
+        butterfly<G::S>(y);
+#pragma unroll
+        for (int t = 0; t < G::S; ++t) {
+            const int j = blk * G::H + c + (t << B);
+            const float z = __fmul_rn(y[t], post);
+            if (kBf16)
+                reinterpret_cast<uint16_t *>(raw)[j] = f32_to_bf16(z);
+            else
+                reinterpret_cast<float *>(raw)[j] = z;
+        }
+    }
+    __syncthreads();
+    copy_out(static_cast<unsigned char *>(out) + row * (int64_t)d * esz, raw, d * esz);
+}
+
+// ---------------------------------------------------------------------------------------------
+// rpbh_quantize_weight: _quantize_rows
+// ---------------------------------------------------------------------------------------------
+struct Edges {
+    float e[15];  // (c_k + c_{k+1}) / 2
+};
+
+__device__ __forceinline__ double block_sum_f64(double v, double *red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double t = 0.0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t = __dadd_rn(t, red[w]);
+        red[32] = t;
+    }
+    __syncthreads();
+    return red[32];
+}
+
+// bucketize(u, edges, right=False): the number of edges strictly below u.
+// kSym: the codebook is antisymmetric (c_k = -c_{L-1-k}), so the middle edge is 0 and the other
+// edges come in +- pairs: count the positive edges below a' = |u| for u > 0, or below
+// a' = next(|u|) for u < 0 (fma with upward rounding: |u| - u 2^-24 rounded up), which turns the
+// "<=" a negative value needs into a strict compare. Otherwise every edge is compared directly.
+template <int BITS, bool kSym>
+__device__ __forceinline__ uint32_t bucketize(float u, const Edges &E) {
+    constexpr int L = 1 << BITS;
+    if (kSym) {
+        constexpr int mid = L / 2 - 1;
+        const float ap = __fmaf_ru(u, -0x1p-24f, fabsf(u));
+        uint32_t c = 0;
+#pragma unroll
+        for (int k = mid + 1; k < L - 1; ++k) c += (uint32_t)(ap > E.e[k]);
+        return u > 0.0f ? (uint32_t)(mid + 1) + c : (uint32_t)mid - c;
+    } else {
+        uint32_t c = 0;
+#pragma unroll
+        for (int k = 0; k < L - 1; ++k) c += (uint32_t)(u > E.e[k]);
+        return c;
+    }
+}
+
+template <int B, bool kBf16, int BITS, bool kSym>
+__global__ void __launch_bounds__(kMaxThreads)
+    quantize_kernel(const void *__restrict__ w, int d, float post, const int32_t *__restrict__ perm,
+                    const int8_t *__restrict__ signs, Edges E, uint8_t *__restrict__ packed,
+                    void *__restrict__ row_norms) {
+    using G = Geo<B>;
+    constexpr int esz = kBf16 ? 2 : 4;
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ double red[33];
+    unsigned char *raw = align16(smem_raw);
+    unsigned char *buf = raw + (size_t)d * esz;
+    const int64_t row = blockIdx.x;
+    copy_in(raw, static_cast<const unsigned char *>(w) + row * (int64_t)d * esz, d * esz);
+    __syncthreads();
+    const int nslots = d >> B;
+    for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+        const int blk = s >> B, r = s & (G::S - 1);
+        float y[G::S];
+        gather_row<B, kBf16>(y, raw, blk * G::H + r * G::S, d, perm, signs);
+        store_row<B>(buf, y, blk, r);
+    }
+    __syncthreads();
+    // pass 1: w_rot = fwht * h^-0.5, written back in place; fp64 sum of exact squares
+    double ss = 0.0;
+    float *fb = reinterpret_cast<float *>(buf);
+    for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+        const int blk = s >> B, c = s & (G::S - 1);
+        float y[G::S];
+        load_col<B>(y, buf, blk, c);
+        butterfly<G::S>(y);
+#pragma unroll
+        for (int t = 0; t < G::S; ++t) {
+            const float z = __fmul_rn(y[t], post);
+            fb[bufpos<B>(blk, t, c)] = z;
+            const double dz = (double)z;
+            ss = __fma_rn(dz, dz, ss);
+        }
+    }
+    // rho = ||w_rot||; unit = w_rot / (rho + 1e-10)
+    const float rho = __double2float_rn(__dsqrt_rn(block_sum_f64(ss, red)));
+    const float den = __fadd_rn(rho, 1e-10f);
+    const float rden = __frcp_rn(den);
+    for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+        const int blk = s >> B, c = s & (G::S - 1);
+#pragma unroll
+        for (int t = 0; t < G::S; ++t) {
+            const float z = fb[bufpos<B>(blk, t, c)];
+            // correctly rounded z / den (Markstein: r = RN(1/den), q0 = RN(z r), e exact, RN(q0 + e r))
+            const float q0 = __fmul_rn(z, rden);
+            const float u = __fmaf_rn(__fmaf_rn(-q0, den, z), rden, q0);
+            raw[blk * G::H + c + (t << B)] = (uint8_t)bucketize<BITS, kSym>(u, E);
+        }
+    }
+    __syncthreads();
+    // pack_codes: 32 codes -> BITS big-endian 32-bit words of the MSB-first stream
+    uint8_t *dst = packed + (row * (int64_t)d / 8) * BITS;
+    for (int g = threadIdx.x; g < d / 32; g += blockDim.x) {
+        const uint4 c0 = *reinterpret_cast<const uint4 *>(raw + 32 * g);
+        const uint4 c1 = *reinterpret_cast<const uint4 *>(raw + 32 * g + 16);
+        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        unsigned __int128 acc = 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc = (acc << BITS) | ((cw[i >> 2] >> (8 * (i & 3))) & 0xffu);
+#pragma unroll
+        for (int k = 0; k < BITS; ++k) {
+            const uint32_t word = (uint32_t)(acc >> (32 * (BITS - 1 - k)));
+            reinterpret_cast<uint32_t *>(dst + 4 * BITS * g)[k] = __byte_perm(word, 0, 0x0123);
+        }
+    }
+    if (threadIdx.x == 0) {
+        if (kBf16)
+            static_cast<uint16_t *>(row_norms)[row] = f32_to_bf16(rho);
+        else
+            static_cast<float *>(row_norms)[row] = rho;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// rpbh_dequantize_weight with unrotate: _dequantize_rotated(fp32) then rpbh_inverse
+// ---------------------------------------------------------------------------------------------
+struct Codebook {
+    float c[16];
+};
+
+template <int B, bool kNormBf16, bool kOutBf16, int BITS>
+__global__ void __launch_bounds__(kMaxThreads)
+    dequant_unrotate_kernel(const uint8_t *__restrict__ packed, const void *__restrict__ row_norms, int d,
+                            float post, Codebook cb, const int32_t *__restrict__ perm,
+                            const int8_t *__restrict__ signs, void *__restrict__ out) {
+    using G = Geo<B>;
+    constexpr int oesz = kOutBf16 ? 2 : 4;
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ float cbs[16];
+    unsigned char *codes = align16(smem_raw);
+    unsigned char *buf = codes + d;
+    unsigned char *stage = buf + (size_t)d * 4;
+    const int64_t row = blockIdx.x;
+    if (threadIdx.x < (1u << BITS)) cbs[threadIdx.x] = cb.c[threadIdx.x];
+    const float rho = kNormBf16 ? bf16_to_f32(static_cast<const uint16_t *>(row_norms)[row])
+                                : static_cast<const float *>(row_norms)[row];
+    // unpack_codes: BITS big-endian words -> 32 codes
+    const uint8_t *src = packed + (row * (int64_t)d / 8) * BITS;
+    for (int g = threadIdx.x; g < d / 32; g += blockDim.x) {
+        unsigned __int128 acc = 0;
+#pragma unroll
+        for (int k = 0; k < BITS; ++k)
+            acc = (acc << 32) | __byte_perm(__ldg(reinterpret_cast<const uint32_t *>(src + 4 * BITS * g) + k), 0, 0x0123);
+        uint32_t cw[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            uint32_t wv = 0;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int i = 4 * q + b;
+                wv |= (uint32_t)((acc >> (BITS * (31 - i))) & ((1u << BITS) - 1)) << (8 * b);
+            }
+            cw[q] = wv;
+        }
+        *reinterpret_cast<uint4 *>(codes + 32 * g) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        *reinterpret_cast<uint4 *>(codes + 32 * g + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    }
+    __syncthreads();
+    const int nslots = d >> B;
+    for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+        const int blk = s >> B, r = s & (G::S - 1);
+        const int j0 = blk * G::H + r * G::S;
+        float y[G::S];
+#pragma unroll
+        for (int t = 0; t < G::S; ++t) y[t] = __fmul_rn(cbs[codes[j0 + t]], rho);  // W' = codebook[code] * rho
+        butterfly<G::S>(y);
+        store_row<B>(buf, y, blk, r);
+    }
+    __syncthreads();
+    for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+        const int blk = s >> B, c = s & (G::S - 1);
+        float y[G::S];
+        load_col<B>(y, buf, blk, c);
+        butterfly<G::S>(y);
+#pragma unroll
+        for (int t = 0; t < G::S; ++t) {
+            const int j = blk * G::H + c + (t << B);
+            // z = fwht * h^-0.5 * signs; out[perm[j]] = z
+            const float z = __fmul_rn(__fmul_rn(y[t], post), (float)__ldg(signs + j));
+            const int p = clampi(__ldg(perm + j), d);
+            if (kOutBf16)
+                reinterpret_cast<uint16_t *>(stage)[p] = f32_to_bf16(z);
+            else
+                reinterpret_cast<float *>(stage)[p] = z;
+        }
+    }
+    __syncthreads();
+    copy_out(static_cast<unsigned char *>(out) + row * (int64_t)d * oesz, stage, d * oesz);
+}
+
+// ---------------------------------------------------------------------------------------------
+// host dispatch
+// ---------------------------------------------------------------------------------------------
+int log2_block(int64_t d) {
+    const int64_t h = d & -d;
+    int l = 0;
+    while ((int64_t(1) << l) < h) ++l;
+    return l;
+}
+
+size_t smem_limit() {
+    int dev = 0, optin = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+    return (size_t)optin;
+}
+
+size_t rot_smem(int64_t d, int esz) { return (size_t)d * (esz + 4) + 16; }
+size_t deq_smem(int64_t d, int oesz) { return (size_t)d * (1 + 4 + oesz) + 16; }
+
+bool supported(int64_t d, int in_esz, int out_esz) {
+    const int l = log2_block(d);
+    if (l < 6 || l > 12 || (l & 1)) return false;
+    if (d > 65536) return false;
+    const size_t a = rot_smem(d, in_esz > out_esz ? in_esz : out_esz), b = deq_smem(d, out_esz);
+    return (a > b ? a : b) + 2048 <= smem_limit();
+}
+
+int threads_for(int64_t d, int B) {
+    const int64_t slots = d >> B;
+    int64_t t = ((slots + 31) / 32) * 32;
+    if (t > kMaxThreads) t = kMaxThreads;
+    if (t < 64) t = 64;
+    return (int)t;
+}
+
+template <typename K>
+wq_status prep(K k, size_t smem) {
+    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return WQ_ERR_CUDA;
+    return WQ_OK;
+}
+
+float fwht_post(int64_t h) { return (float)std::pow((double)h, -0.5); }
+
+template <int B, bool kBf16>
+wq_status rotate_b(const void *x, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs, void *out,
+                   cudaStream_t s) {
+    const size_t smem = rot_smem(d, kBf16 ? 2 : 4);
+    auto k = rotate_kernel<B, kBf16>;
+    wq_status st = prep(k, smem);
+    if (st != WQ_OK) return st;
+    k<<<(unsigned)rows, threads_for(d, B), smem, s>>>(x, (int)d, fwht_post(d & -d), perm, signs, out);
+    return launch_status();
+}
+
+wq_status rotate(const void *x, int dtype, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
+                 void *out, cudaStream_t s) {
+    const bool bf = dtype == WQ_BF16;
+    switch (log2_block(d) / 2) {
+        case 3: return bf ? rotate_b<3, true>(x, rows, d, perm, signs, out, s) : rotate_b<3, false>(x, rows, d, perm, signs, out, s);
+        case 4: return bf ? rotate_b<4, true>(x, rows, d, perm, signs, out, s) : rotate_b<4, false>(x, rows, d, perm, signs, out, s);
+        case 5: return bf ? rotate_b<5, true>(x, rows, d, perm, signs, out, s) : rotate_b<5, false>(x, rows, d, perm, signs, out, s);
+        case 6: return bf ? rotate_b<6, true>(x, rows, d, perm, signs, out, s) : rotate_b<6, false>(x, rows, d, perm, signs, out, s);
+        default: return WQ_ERR_SHAPE;
+    }
+}
+
+template <int B, bool kBf16, int BITS, bool kSym>
+wq_status quantize_b(const void *w, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
+                     const Edges &E, uint8_t *packed, void *row_norms, cudaStream_t s) {
+    const size_t smem = rot_smem(d, kBf16 ? 2 : 4);
+    auto k = quantize_kernel<B, kBf16, BITS, kSym>;
+    wq_status st = prep(k, smem);
+    if (st != WQ_OK) return st;
+    k<<<(unsigned)rows, threads_for(d, B), smem, s>>>(w, (int)d, fwht_post(d & -d), perm, signs, E, packed, row_norms);
+    return launch_status();
+}
+
+template <int B, bool kBf16, bool kSym>
+wq_status quantize_bits(int bits, const void *w, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
+                        const Edges &E, uint8_t *packed, void *row_norms, cudaStream_t s) {
+    switch (bits) {
+        case 2: return quantize_b<B, kBf16, 2, kSym>(w, rows, d, perm, signs, E, packed, row_norms, s);
+        case 3: return quantize_b<B, kBf16, 3, kSym>(w, rows, d, perm, signs, E, packed, row_norms, s);
+        case 4: return quantize_b<B, kBf16, 4, kSym>(w, rows, d, perm, signs, E, packed, row_norms, s);
+        default: return WQ_ERR_BITS;
+    }
+}
+
+template <int B>
+wq_status quantize_sym(bool bf, bool sym, int bits, const void *w, int64_t rows, int64_t d, const int32_t *perm,
+                       const int8_t *signs, const Edges &E, uint8_t *packed, void *row_norms, cudaStream_t s) {
+    if (bf)
+        return sym ? quantize_bits<B, true, true>(bits, w, rows, d, perm, signs, E, packed, row_norms, s)
+                   : quantize_bits<B, true, false>(bits, w, rows, d, perm, signs, E, packed, row_norms, s);
+    return sym ? quantize_bits<B, false, true>(bits, w, rows, d, perm, signs, E, packed, row_norms, s)
+               : quantize_bits<B, false, false>(bits, w, rows, d, perm, signs, E, packed, row_norms, s);
+}
+
+wq_status quantize(const void *w, int w_dtype, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
+                   int bits, const float *codebook, uint8_t *packed, void *row_norms, cudaStream_t s) {
+    const int L = 1 << bits;
+    Edges E = {};
+    // edges = (codebook[:-1] + codebook[1:]) / 2, in fp32 as the page computes them
+    for (int k = 0; k + 1 < L; ++k) {
+        volatile float sum = codebook[k] + codebook[k + 1];
+        E.e[k] = sum / 2.0f;
+    }
+    bool sym = true;
+    for (int k = 0; k < L; ++k)
+        if (!(codebook[k] == -codebook[L - 1 - k])) sym = false;
+    if (sym && !(E.e[L / 2 - 1] == 0.0f)) sym = false;
+    const bool bf = w_dtype == WQ_BF16;
+    switch (log2_block(d) / 2) {
+        case 3: return quantize_sym<3>(bf, sym, bits, w, rows, d, perm, signs, E, packed, row_norms, s);
+        case 4: return quantize_sym<4>(bf, sym, bits, w, rows, d, perm, signs, E, packed, row_norms, s);
+        case 5: return quantize_sym<5>(bf, sym, bits, w, rows, d, perm, signs, E, packed, row_norms, s);
+        case 6: return quantize_sym<6>(bf, sym, bits, w, rows, d, perm, signs, E, packed, row_norms, s);
+        default: return WQ_ERR_SHAPE;
+    }
+}
+
+template <int B, bool kNB, bool kOB, int BITS>
+wq_status deq_b(const uint8_t *packed, const void *norms, int64_t rows, int64_t d, const Codebook &cb,
+                const int32_t *perm, const int8_t *signs, void *out, cudaStream_t s) {
+    const size_t smem = deq_smem(d, kOB ? 2 : 4);
+    auto k = dequant_unrotate_kernel<B, kNB, kOB, BITS>;
+    wq_status st = prep(k, smem);
+    if (st != WQ_OK) return st;
+    k<<<(unsigned)rows, threads_for(d, B), smem, s>>>(packed, norms, (int)d, fwht_post(d & -d), cb, perm, signs, out);
+    return launch_status();
+}
+
+template <int B, bool kNB, bool kOB>
+wq_status deq_bits(int bits, const uint8_t *packed, const void *norms, int64_t rows, int64_t d, const Codebook &cb,
+                   const int32_t *perm, const int8_t *signs, void *out, cudaStream_t s) {
+    switch (bits) {
+        case 2: return deq_b<B, kNB, kOB, 2>(packed, norms, rows, d, cb, perm, signs, out, s);
+        case 3: return deq_b<B, kNB, kOB, 3>(packed, norms, rows, d, cb, perm, signs, out, s);
+        case 4: return deq_b<B, kNB, kOB, 4>(packed, norms, rows, d, cb, perm, signs, out, s);
+        default: return WQ_ERR_BITS;
+    }
+}
+
+template <int B>
+wq_status deq_dt(bool nb, bool ob, int bits, const uint8_t *packed, const void *norms, int64_t rows, int64_t d,
+                 const Codebook &cb, const int32_t *perm, const int8_t *signs, void *out, cudaStream_t s) {
+    if (nb)
+        return ob ? deq_bits<B, true, true>(bits, packed, norms, rows, d, cb, perm, signs, out, s)
+                  : deq_bits<B, true, false>(bits, packed, norms, rows, d, cb, perm, signs, out, s);
+    return ob ? deq_bits<B, false, true>(bits, packed, norms, rows, d, cb, perm, signs, out, s)
+              : deq_bits<B, false, false>(bits, packed, norms, rows, d, cb, perm, signs, out, s);
+}
+
+wq_status dequantize_unrotate(const uint8_t *packed, const void *row_norms, int norm_dtype, int64_t rows, int64_t d,
+                              int bits, const float *codebook, const int32_t *perm, const int8_t *signs, void *out,
+                              int out_dtype, cudaStream_t s) {
+    Codebook cb = {};
+    for (int k = 0; k < (1 << bits); ++k) cb.c[k] = codebook[k];
+    const bool nb = norm_dtype == WQ_BF16, ob = out_dtype == WQ_BF16;
+    switch (log2_block(d) / 2) {
+        case 3: return deq_dt<3>(nb, ob, bits, packed, row_norms, rows, d, cb, perm, signs, out, s);
+        case 4: return deq_dt<4>(nb, ob, bits, packed, row_norms, rows, d, cb, perm, signs, out, s);
+        case 5: return deq_dt<5>(nb, ob, bits, packed, row_norms, rows, d, cb, perm, signs, out, s);
+        case 6: return deq_dt<6>(nb, ob, bits, packed, row_norms, rows, d, cb, perm, signs, out, s);
+        default: return WQ_ERR_SHAPE;
+    }
+}
+
+}  // namespace rpbh_fast
+}  // namespace wq

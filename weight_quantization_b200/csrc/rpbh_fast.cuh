@@ -1,0 +1,28 @@
+// Register-blocked RPBH kernels (see rpbh_fast.cu). Internal interface between the C ABI in
+// rpbh.cu and the fast kernels; not part of the exported library surface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "wq.h"
+
+namespace wq {
+namespace rpbh_fast {
+
+// True when the fast kernels handle this (d, dtype) pair: Hadamard block h = d & -d with an even
+// log2 between 6 and 12 (h = 64, 256, 1024, 4096) and a row that fits in shared memory.
+bool supported(int64_t d, int in_esz, int out_esz);
+
+wq_status rotate(const void *x, int dtype, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
+                 void *out, cudaStream_t s);
+
+wq_status quantize(const void *w, int w_dtype, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
+                   int bits, const float *codebook, uint8_t *packed, void *row_norms, cudaStream_t s);
+
+wq_status dequantize_unrotate(const uint8_t *packed, const void *row_norms, int norm_dtype, int64_t rows, int64_t d,
+                              int bits, const float *codebook, const int32_t *perm, const int8_t *signs, void *out,
+                              int out_dtype, cudaStream_t s);
+
+}  // namespace rpbh_fast
+}  // namespace wq
