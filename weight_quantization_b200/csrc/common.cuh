@@ -53,6 +53,11 @@ inline wq_status launch_status() {
 }
 
 inline bool valid_dtype(int t) { return t == WQ_F32 || t == WQ_BF16; }
+
+// Raise a kernel's dynamic shared-memory limit to `smem` bytes the first time a call needs more
+// than the current setting (tracked per kernel and device), so that later calls -- including
+// calls made while a stream is captured into a CUDA graph -- issue no attribute change.
+bool ensure_dynamic_smem(const void *kernel, size_t smem);
 inline int dtype_size(int t) { return t == WQ_F32 ? 4 : 2; }
 
 }  // namespace wq

@@ -221,18 +221,25 @@ inline wq_status check_dims(int64_t rows, int64_t d) {
     return WQ_OK;
 }
 
-// Opt in to more than 48 KB of dynamic shared memory when a row needs it.
+// Opt in to more than 48 KB of dynamic shared memory when a row needs it. The attribute is set
+// once per kernel (and again only if a later call needs more), so calls made while a stream is
+// being captured into a CUDA graph issue no attribute changes.
+inline size_t optin_limit() {
+    static size_t cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (!cached[dev]) {
+        int optin = 0;
+        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+        cached[dev] = (size_t)optin;
+    }
+    return cached[dev];
+}
+
 template <typename K>
 inline wq_status prepare(K kernel, size_t smem) {
-    int dev = 0, optin = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return WQ_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-        return WQ_ERR_CUDA;
-    if (smem + 1024 > (size_t)optin) return WQ_ERR_SHAPE;
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return WQ_ERR_CUDA;
-    return WQ_OK;
+    if (smem + 1024 > optin_limit()) return WQ_ERR_SHAPE;
+    return ensure_dynamic_smem(reinterpret_cast<const void *>(kernel), smem) ? WQ_OK : WQ_ERR_CUDA;
 }
 
 }  // namespace rpbh

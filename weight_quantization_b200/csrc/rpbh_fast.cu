@@ -393,10 +393,15 @@ int log2_block(int64_t d) {
 }
 
 size_t smem_limit() {
-    int dev = 0, optin = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
-    return (size_t)optin;
+    static size_t cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (!cached[dev]) {
+        int optin = 0;
+        if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+        cached[dev] = (size_t)optin;
+    }
+    return cached[dev];
 }
 
 size_t rot_smem(int64_t d, int esz) { return (size_t)d * (esz + 4) + 16; }
@@ -418,11 +423,10 @@ int threads_for(int64_t d, int B) {
     return (int)t;
 }
 
+// Raise a kernel's dynamic shared-memory limit once (and again only when a call needs more).
 template <typename K>
 wq_status prep(K k, size_t smem) {
-    if (smem > 48 * 1024 && cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return WQ_ERR_CUDA;
-    return WQ_OK;
+    return ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem) ? WQ_OK : WQ_ERR_CUDA;
 }
 
 float fwht_post(int64_t h) { return (float)std::pow((double)h, -0.5); }

@@ -5,7 +5,9 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <map>
 #include <mutex>
+#include <utility>
 
 namespace wq {
 
@@ -40,6 +42,21 @@ bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, ui
     return fn(map, dt, 2, const_cast<void *>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool ensure_dynamic_smem(const void *kernel, size_t smem) {
+    if (smem <= 48 * 1024) return true;
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, size_t> set_to;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    std::lock_guard<std::mutex> lock(mu);
+    size_t &cur = set_to[std::make_pair(kernel, dev)];
+    if (smem <= cur) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return false;
+    cur = smem;
+    return true;
 }
 
 }  // namespace wq
