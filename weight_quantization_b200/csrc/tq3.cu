@@ -16,7 +16,9 @@
 //     r = RN(1/d), q0 = RN(x r), e = x - q0 d (exact by FMA), RN(q0 + e r) = RN(x / d)
 //     (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000 processor",
 //     IBM J. Res. Dev. 34(1), 1990); it is checked bit for bit against IEEE division by the tests;
-//   * the butterflies and post-multipliers are single IEEE additions and multiplications.
+//   * the butterflies and post-multipliers are single IEEE additions and multiplications (the
+//     last stage as one fused a * (+-1) + b, which rounds once like an addition);
+//   * the indices come from exact 0/1 saturated steps summed on the FMA pipe (add_index).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -65,6 +67,36 @@ __device__ __forceinline__ uint32_t pair_flip(int k, uint32_t H, uint32_t mlo, u
     }
 }
 
+// Encoder split of the flips: with the page's table the half-0 pattern C0 is applied later as
+// operand negation in the first butterfly stage, so the words only take (C0 ^ C1) for half 1;
+// any other table takes the whole pattern on the words.
+template <bool kDefault>
+__device__ __forceinline__ uint32_t word_flip(int k, uint32_t H, uint32_t mlo, uint32_t mhi) {
+    if (kDefault) {
+        const uint32_t c0 = (default_flip(2 * k) >> 16) | default_flip(2 * k + 1);
+        const uint32_t c1 = (default_flip(64 + 2 * k) >> 16) | default_flip(64 + 2 * k + 1);
+        return H & (c0 ^ c1);
+    }
+    return pair_flip<false>(k, H, mlo, mhi);
+}
+template <bool kDefault>
+__host__ __device__ constexpr bool stage1_neg(int e) {
+    return kDefault && default_flip(e) != 0;
+}
+
+// Stage h = 64: element i (half 0) with element i + 64 (half 1). Half 0 keeps a + o and half 1
+// keeps o - a, both as one rounding of a * (+-1) + o.
+__device__ __forceinline__ void stage64(float (&a)[64], int half) {
+    const float sg = half ? -1.0f : 1.0f;
+    const f32x2 S = pk2(sg, sg);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+        const float o0 = __shfl_xor_sync(0xffffffffu, a[2 * k], 16);
+        const float o1 = __shfl_xor_sync(0xffffffffu, a[2 * k + 1], 16);
+        upk2(fma2(pk2(a[2 * k], a[2 * k + 1]), S, pk2(o0, o1)), a[2 * k], a[2 * k + 1]);
+    }
+}
+
 // fp32(1.0 / math.sqrt(128)), the post-multiplier of _fwht_inplace.
 __device__ __forceinline__ float fwht_post() { return __uint_as_float(0x3DB504F3u); }
 
@@ -75,19 +107,22 @@ __device__ __forceinline__ f32x2 div2(f32x2 x, f32x2 r, f32x2 neg_d) {
     return fma2(e, r, q0);
 }
 
-// searchsorted(TQ3_BOUNDARIES, q, right=False) as a sum of exact 0/1 steps [q > B_j] computed on
-// the FMA pipe: for |B_j| >= 0.2304 any fp32 q above B_j exceeds it by at least 2^-26, so
-// (q - B_j) * 2^26 >= 1 and the saturated value is exactly 1; q <= B_j saturates to 0. The step at
-// B = 0 scales twice so that the smallest subnormal q > 0 still reaches 1.
-__device__ __forceinline__ float bucket_steps(float q) {
+// Adds 8^i * idx to the fp32 group word, idx = searchsorted(TQ3_BOUNDARIES, q, right=False), the
+// number of boundaries strictly below q. With a' = RU(|q| - q 2^-24) -- |q| for q > 0 (or the
+// float just below it when q is a power of two, which no boundary sits next to) and next(|q|) for
+// q < 0 -- the count of positive boundaries b with b < a' is c = #{b < q} for q > 0 and
+// c = #{b <= |q|} for q < 0, so idx = 4 + c for q > 0 and idx = 3 - c otherwise (q = +-0 gives
+// a' = 0 and idx 3). Each [b < a'] is an exact 0/1: a' and b are floats of magnitude >= 2^-3,
+// so a' > b implies (a' - b) 2^26 >= 1 and the saturated value is 1; a' <= b saturates to 0.
+// Every term is an integer below 2^24, so the word is exact.
+__device__ __forceinline__ float add_index(float q, float w8, float word) {
+    const float ap = __fmaf_ru(q, -0x1p-24f, fabsf(q));
     const float M = 67108864.0f;  // 2^26
-    float t = __saturatef(__fmaf_rn(q, M, 0.7992f * M)) + __saturatef(__fmaf_rn(q, M, 0.4824f * M));
-    t = t + __saturatef(__fmaf_rn(q, M, 0.2304f * M));
-    t = t + __saturatef(__fmul_rn(__saturatef(__fmul_rn(q, 0x1p100f)), 0x1p100f));
-    t = t + __saturatef(__fmaf_rn(q, M, -0.2304f * M));
-    t = t + __saturatef(__fmaf_rn(q, M, -0.4824f * M));
-    t = t + __saturatef(__fmaf_rn(q, M, -0.7992f * M));
-    return t;
+    float c = __saturatef(__fmaf_rn(ap, M, -0.2304f * M));
+    c = __fadd_rn(c, __saturatef(__fmaf_rn(ap, M, -0.4824f * M)));
+    c = __fadd_rn(c, __saturatef(__fmaf_rn(ap, M, -0.7992f * M)));
+    const bool pos = q > 0.0f;
+    return __fmaf_rn(pos ? w8 : -w8, c, __fadd_rn(word, pos ? 4.0f * w8 : 3.0f * w8));
 }
 
 // TQ3_CENTROIDS as printed on the page (fp32).
@@ -165,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const int k = 4 * j + u;
-                const uint32_t w = w4[u] ^ pair_flip<kDefault>(k, H, mlo, mhi);
+                const uint32_t w = w4[u] ^ word_flip<kDefault>(k, H, mlo, mhi);
                 x[2 * k] = bf16_lo(w);
                 x[2 * k + 1] = bf16_hi(w);
             }
@@ -179,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 #pragma unroll
             for (int u = 0; u < 4; u += 2) {
                 const int k = 2 * j + u / 2;
-                const uint32_t f = pair_flip<kDefault>(k, H, mlo, mhi);
+                const uint32_t f = word_flip<kDefault>(k, H, mlo, mhi);
                 x[2 * k] = __uint_as_float(w4[u] ^ (f << 16));
                 x[2 * k + 1] = __uint_as_float(w4[u + 1] ^ (f & 0x80000000u));
             }
@@ -205,19 +240,16 @@ __global__ void __launch_bounds__(kThreads, 4)
 #pragma unroll
         for (int k = 0; k < 32; ++k) upk2(div2(pk2(x[2 * k], x[2 * k + 1]), R, ND), a[2 * k], a[2 * k + 1]);
     }
+    // stage 1, with the rest of the default-table flips as (exact) operand negations
 #pragma unroll
     for (int k = 0; k < 32; ++k) {
-        const float p = a[2 * k], q = a[2 * k + 1];
+        const float p = stage1_neg<kDefault>(2 * k) ? -a[2 * k] : a[2 * k];
+        const float q = stage1_neg<kDefault>(2 * k + 1) ? -a[2 * k + 1] : a[2 * k + 1];
         a[2 * k] = __fadd_rn(p, q);
         a[2 * k + 1] = __fsub_rn(p, q);
     }
     fwht_local_2_32(a);
-    // stage h = 64: element i (half 0) with element i + 64 (half 1)
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, a[i], 16);
-        a[i] = half ? __fsub_rn(o, a[i]) : __fadd_rn(a[i], o);
-    }
+    stage64(a, half);
 
     // Step 4: scale = max(max|xh|, 1e-8) with xh = fwht * c; max|fl(y c)| = fl(max|y| c)
     float m = 0.0f;
@@ -239,8 +271,8 @@ __global__ void __launch_bounds__(kThreads, 4)
             for (int i = 0; i < 8; i += 2) {
                 float q0, q1;
                 upk2(div2(mul2(pk2(a[8 * g + i], a[8 * g + i + 1]), C2), RS, NS), q0, q1);
-                wf = __fmaf_rn(bucket_steps(q0), (float)(1u << (3 * i)), wf);
-                wf = __fmaf_rn(bucket_steps(q1), (float)(1u << (3 * i + 3)), wf);
+                wf = add_index(q0, (float)(1u << (3 * i)), wf);
+                wf = add_index(q1, (float)(1u << (3 * i + 3)), wf);
             }
             grp[g] = __float2uint_rz(wf);  // exact: an integer below 2^24
         }
