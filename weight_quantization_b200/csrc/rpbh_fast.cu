@@ -383,6 +383,253 @@ __global__ void __launch_bounds__(kMaxThreads)
 }
 
 // ---------------------------------------------------------------------------------------------
+// Persistent variants: each CTA keeps the permutation (16-bit) and the sign bits in shared memory
+// and walks rows blockIdx.x, blockIdx.x + gridDim.x, ...; the next row is fetched with a 1-D bulk
+// copy into the other of two row buffers while the current row is processed.
+// ---------------------------------------------------------------------------------------------
+constexpr uint32_t kMaxPolls = 1u << 24;
+__device__ unsigned int g_fault;
+
+__host__ __device__ constexpr int a16(int x) { return (x + 15) & ~15; }
+
+struct PLayout {
+    int perm, bits, row0, row1, buf, bar, total;
+    __host__ __device__ PLayout(int d, int esz) {
+        perm = 0;
+        bits = a16(2 * d);
+        row0 = bits + a16(d / 8);
+        row1 = row0 + d * esz;
+        buf = row1 + d * esz;
+        bar = buf + 4 * d;
+        total = bar + 16;
+    }
+};
+
+// Tables into shared memory: perm as 16-bit indices (clamped into the row), signs as bits
+// (bit t of word w set when signs[32 w + t] is negative).
+__device__ __forceinline__ void load_tables(uint16_t *perm16, uint32_t *sbits, const int32_t *__restrict__ perm,
+                                            const int8_t *__restrict__ signs, int d) {
+    for (int j = threadIdx.x; j < d; j += blockDim.x) perm16[j] = (uint16_t)clampi(__ldg(perm + j), d);
+    for (int w = threadIdx.x; w < d / 32; w += blockDim.x) {
+        uint32_t bits = 0;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int4 v = __ldg(reinterpret_cast<const int4 *>(signs + 32 * w) + q);
+            const uint32_t wv[4] = {(uint32_t)v.x, (uint32_t)v.y, (uint32_t)v.z, (uint32_t)v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) bits |= ((wv[u] >> (8 * b + 7)) & 1u) << (16 * q + 4 * u + b);
+        }
+        sbits[w] = bits;
+    }
+}
+
+// pass 0 from the staged row: y[t] = x[perm[j0 + t]] * signs[j0 + t] (the sign as a bit flip)
+template <int B, bool kBf16>
+__device__ __forceinline__ void gather_row_smem(float (&y)[1 << B], const unsigned char *raw, int j0,
+                                                const uint16_t *perm16, const uint32_t *sbits) {
+    constexpr int S = 1 << B;
+    uint32_t pw[S / 2];
+#pragma unroll
+    for (int q = 0; q < S / 8; ++q) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(perm16 + j0 + 8 * q);
+        pw[4 * q] = v.x; pw[4 * q + 1] = v.y; pw[4 * q + 2] = v.z; pw[4 * q + 3] = v.w;
+    }
+    uint32_t sw[(S + 31) / 32];
+#pragma unroll
+    for (int q = 0; q < (S + 31) / 32; ++q) sw[q] = sbits[(j0 >> 5) + q] >> (S < 32 ? (j0 & 31) : 0);
+#pragma unroll
+    for (int t = 0; t < S; ++t) {
+        const uint32_t p = (pw[t >> 1] >> (16 * (t & 1))) & 0xffffu;
+        const uint32_t flip = ((sw[t >> 5] >> (t & 31)) & 1u) << 31;
+        const uint32_t xb = kBf16 ? (uint32_t)reinterpret_cast<const uint16_t *>(raw)[p] << 16
+                                  : reinterpret_cast<const uint32_t *>(raw)[p];
+        y[t] = __uint_as_float(xb ^ flip);
+    }
+    butterfly<S>(y);
+}
+
+// Waits for this row's bulk copy; if the bounded wait runs out anywhere in the CTA, every thread
+// learns it (so no thread is left at a later barrier), the fault flag is set and the caller stops.
+__device__ __forceinline__ bool row_ready(uint64_t *bar, uint32_t parity) {
+    const bool ok = mbar_wait_bounded(bar, parity, kMaxPolls);
+    const bool any_fail = __syncthreads_or(!ok);
+    if (any_fail && threadIdx.x == 0) atomicOr(&g_fault, 2u);
+    return !any_fail;
+}
+
+template <int B, bool kBf16>
+__global__ void __launch_bounds__(kMaxThreads)
+    rotate_persistent(const void *__restrict__ x, int rows, int d, float post, const int32_t *__restrict__ perm,
+                      const int8_t *__restrict__ signs, void *__restrict__ out) {
+    using G = Geo<B>;
+    constexpr int esz = kBf16 ? 2 : 4;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = align16(smem_raw);
+    const PLayout Lo(d, esz);
+    uint16_t *perm16 = reinterpret_cast<uint16_t *>(base + Lo.perm);
+    uint32_t *sbits = reinterpret_cast<uint32_t *>(base + Lo.bits);
+    unsigned char *const rb0 = base + Lo.row0;  // row buffers rb0 and rb0 + row_bytes
+    unsigned char *buf = base + Lo.buf;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + Lo.bar);
+    const uint32_t row_bytes = (uint32_t)d * esz;
+    load_tables(perm16, sbits, perm, signs, d);
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+    }
+    __syncthreads();
+    const unsigned char *xb = static_cast<const unsigned char *>(x);
+    int row = blockIdx.x;
+    if (threadIdx.x == 0 && row < rows) {
+        mbar_expect_tx(&bar[0], row_bytes);
+        bulk_load(rb0, xb + (int64_t)row * row_bytes, row_bytes, &bar[0]);
+    }
+    const int nslots = d >> B;
+    for (int it = 0; row < rows; ++it, row += gridDim.x) {
+        const int cur = it & 1;
+        const int nrow = row + gridDim.x;
+        if (threadIdx.x == 0 && nrow < rows) {
+            mbar_expect_tx(&bar[cur ^ 1], row_bytes);
+            bulk_load((rb0 + (cur ^ 1) * row_bytes), xb + (int64_t)nrow * row_bytes, row_bytes, &bar[cur ^ 1]);
+        }
+        if (!row_ready(&bar[cur], (it >> 1) & 1)) {
+            if (threadIdx.x == 0 && nrow < rows) mbar_wait_bounded(&bar[cur ^ 1], ((it + 1) >> 1) & 1, kMaxPolls);
+            return;
+        }
+        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+            const int blk = s >> B, r = s & (G::S - 1);
+            float y[G::S];
+            gather_row_smem<B, kBf16>(y, (rb0 + cur * row_bytes), blk * G::H + r * G::S, perm16, sbits);
+            store_row<B>(buf, y, blk, r);
+        }
+        __syncthreads();
+        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+            const int blk = s >> B, c = s & (G::S - 1);
+            float y[G::S];
+            load_col<B>(y, buf, blk, c);
+            butterfly<G::S>(y);
+#pragma unroll
+            for (int t = 0; t < G::S; ++t) {
+                const int j = blk * G::H + c + (t << B);
+                const float z = __fmul_rn(y[t], post);
+                if (kBf16)
+                    reinterpret_cast<uint16_t *>((rb0 + cur * row_bytes))[j] = f32_to_bf16(z);
+                else
+                    reinterpret_cast<float *>((rb0 + cur * row_bytes))[j] = z;
+            }
+        }
+        __syncthreads();
+        copy_out(static_cast<unsigned char *>(out) + (int64_t)row * row_bytes, (rb0 + cur * row_bytes), row_bytes);
+        fence_proxy_async_smem();  // these generic accesses precede the bulk copy that reuses (rb0 + cur * row_bytes)
+        __syncthreads();
+    }
+}
+
+template <int B, bool kBf16, int BITS, bool kSym>
+__global__ void __launch_bounds__(kMaxThreads)
+    quantize_persistent(const void *__restrict__ w, int rows, int d, float post, const int32_t *__restrict__ perm,
+                        const int8_t *__restrict__ signs, Edges E, uint8_t *__restrict__ packed,
+                        void *__restrict__ row_norms) {
+    using G = Geo<B>;
+    constexpr int esz = kBf16 ? 2 : 4;
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ double red[33];
+    unsigned char *base = align16(smem_raw);
+    const PLayout Lo(d, esz);
+    uint16_t *perm16 = reinterpret_cast<uint16_t *>(base + Lo.perm);
+    uint32_t *sbits = reinterpret_cast<uint32_t *>(base + Lo.bits);
+    unsigned char *const rb0 = base + Lo.row0;  // row buffers rb0 and rb0 + row_bytes
+    unsigned char *buf = base + Lo.buf;
+    float *fb = reinterpret_cast<float *>(buf);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + Lo.bar);
+    const uint32_t row_bytes = (uint32_t)d * esz;
+    load_tables(perm16, sbits, perm, signs, d);
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+    }
+    __syncthreads();
+    const unsigned char *wb = static_cast<const unsigned char *>(w);
+    int row = blockIdx.x;
+    if (threadIdx.x == 0 && row < rows) {
+        mbar_expect_tx(&bar[0], row_bytes);
+        bulk_load(rb0, wb + (int64_t)row * row_bytes, row_bytes, &bar[0]);
+    }
+    const int nslots = d >> B;
+    for (int it = 0; row < rows; ++it, row += gridDim.x) {
+        const int cur = it & 1;
+        const int nrow = row + gridDim.x;
+        if (threadIdx.x == 0 && nrow < rows) {
+            mbar_expect_tx(&bar[cur ^ 1], row_bytes);
+            bulk_load((rb0 + (cur ^ 1) * row_bytes), wb + (int64_t)nrow * row_bytes, row_bytes, &bar[cur ^ 1]);
+        }
+        if (!row_ready(&bar[cur], (it >> 1) & 1)) {
+            if (threadIdx.x == 0 && nrow < rows) mbar_wait_bounded(&bar[cur ^ 1], ((it + 1) >> 1) & 1, kMaxPolls);
+            return;
+        }
+        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+            const int blk = s >> B, r = s & (G::S - 1);
+            float y[G::S];
+            gather_row_smem<B, kBf16>(y, (rb0 + cur * row_bytes), blk * G::H + r * G::S, perm16, sbits);
+            store_row<B>(buf, y, blk, r);
+        }
+        __syncthreads();
+        double ss = 0.0;
+        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+            const int blk = s >> B, c = s & (G::S - 1);
+            float y[G::S];
+            load_col<B>(y, buf, blk, c);
+            butterfly<G::S>(y);
+#pragma unroll
+            for (int t = 0; t < G::S; ++t) {
+                const float z = __fmul_rn(y[t], post);
+                fb[bufpos<B>(blk, t, c)] = z;
+                const double dz = (double)z;
+                ss = __fma_rn(dz, dz, ss);
+            }
+        }
+        const float rho = __double2float_rn(__dsqrt_rn(block_sum_f64(ss, red)));
+        const float den = __fadd_rn(rho, 1e-10f);
+        const float rden = __frcp_rn(den);
+        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
+            const int blk = s >> B, c = s & (G::S - 1);
+#pragma unroll
+            for (int t = 0; t < G::S; ++t) {
+                const float z = fb[bufpos<B>(blk, t, c)];
+                const float q0 = __fmul_rn(z, rden);
+                const float u = __fmaf_rn(__fmaf_rn(-q0, den, z), rden, q0);
+                (rb0 + cur * row_bytes)[blk * G::H + c + (t << B)] = (uint8_t)bucketize<BITS, kSym>(u, E);
+            }
+        }
+        __syncthreads();
+        uint8_t *dst = packed + ((int64_t)row * d / 8) * BITS;
+        for (int g = threadIdx.x; g < d / 32; g += blockDim.x) {
+            const uint4 c0 = *reinterpret_cast<const uint4 *>((rb0 + cur * row_bytes) + 32 * g);
+            const uint4 c1 = *reinterpret_cast<const uint4 *>((rb0 + cur * row_bytes) + 32 * g + 16);
+            const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            unsigned __int128 acc = 0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc = (acc << BITS) | ((cw[i >> 2] >> (8 * (i & 3))) & 0xffu);
+#pragma unroll
+            for (int k = 0; k < BITS; ++k) {
+                const uint32_t word = (uint32_t)(acc >> (32 * (BITS - 1 - k)));
+                reinterpret_cast<uint32_t *>(dst + 4 * BITS * g)[k] = __byte_perm(word, 0, 0x0123);
+            }
+        }
+        if (threadIdx.x == 0) {
+            if (kBf16)
+                static_cast<uint16_t *>(row_norms)[row] = f32_to_bf16(rho);
+            else
+                static_cast<float *>(row_norms)[row] = rho;
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
 // host dispatch
 // ---------------------------------------------------------------------------------------------
 int log2_block(int64_t d) {
@@ -419,7 +666,7 @@ int threads_for(int64_t d, int B) {
     const int64_t slots = d >> B;
     int64_t t = ((slots + 31) / 32) * 32;
     if (t > kMaxThreads) t = kMaxThreads;
-    if (t < 64) t = 64;
+    if (t < 128) t = 128;
     return (int)t;
 }
 
@@ -431,14 +678,64 @@ wq_status prep(K k, size_t smem) {
 
 float fwht_post(int64_t h) { return (float)std::pow((double)h, -0.5); }
 
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (!cached[dev]) cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev);
+    return cached[dev];
+}
+
+size_t pers_smem(int64_t d, int esz) { return (size_t)PLayout((int)d, esz).total + 16; }
+
+bool persistent_fits(int64_t d, int esz) { return d <= 32768 && pers_smem(d, esz) + 1024 <= smem_limit(); }
+
+int blocks_per_sm(const void *k, int threads, size_t smem) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess) return 0;
+    return n;
+}
+
+// The persistent form pays for its resident tables with shared memory; it is taken only when that
+// costs no resident CTAs per SM against the one-row-per-CTA form (its extra smem otherwise lowers
+// the number of rows in flight, which is what keeps HBM busy here).
+template <typename KP, typename KR>
+bool prefer_persistent(KP kp, size_t pers, KR kr, size_t plain, int threads) {
+    const int a = blocks_per_sm(reinterpret_cast<const void *>(kp), threads, pers);
+    const int b = blocks_per_sm(reinterpret_cast<const void *>(kr), threads, plain);
+    return a >= 1 && a >= b;
+}
+
+// Grid for a persistent kernel: every SM gets as many CTAs as fit, but never more CTAs than rows.
+template <typename K>
+int persistent_grid(K k, int threads, size_t smem, int64_t rows) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    const int64_t g = (int64_t)per_sm * sm_count();
+    return (int)(g < rows ? g : rows);
+}
+
 template <int B, bool kBf16>
 wq_status rotate_b(const void *x, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs, void *out,
                    cudaStream_t s) {
+    const int threads = threads_for(d, B);
     const size_t smem = rot_smem(d, kBf16 ? 2 : 4);
     auto k = rotate_kernel<B, kBf16>;
     wq_status st = prep(k, smem);
     if (st != WQ_OK) return st;
-    k<<<(unsigned)rows, threads_for(d, B), smem, s>>>(x, (int)d, fwht_post(d & -d), perm, signs, out);
+    if (persistent_fits(d, kBf16 ? 2 : 4)) {
+        const size_t psmem = pers_smem(d, kBf16 ? 2 : 4);
+        auto kp = rotate_persistent<B, kBf16>;
+        st = prep(kp, psmem);
+        if (st != WQ_OK) return st;
+        if (prefer_persistent(kp, psmem, k, smem, threads)) {
+            kp<<<persistent_grid(kp, threads, psmem, rows), threads, psmem, s>>>(x, (int)rows, (int)d,
+                                                                                 fwht_post(d & -d), perm, signs, out);
+            return launch_status();
+        }
+    }
+    k<<<(unsigned)rows, threads, smem, s>>>(x, (int)d, fwht_post(d & -d), perm, signs, out);
     return launch_status();
 }
 
@@ -457,11 +754,23 @@ wq_status rotate(const void *x, int dtype, int64_t rows, int64_t d, const int32_
 template <int B, bool kBf16, int BITS, bool kSym>
 wq_status quantize_b(const void *w, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
                      const Edges &E, uint8_t *packed, void *row_norms, cudaStream_t s) {
+    const int threads = threads_for(d, B);
     const size_t smem = rot_smem(d, kBf16 ? 2 : 4);
     auto k = quantize_kernel<B, kBf16, BITS, kSym>;
     wq_status st = prep(k, smem);
     if (st != WQ_OK) return st;
-    k<<<(unsigned)rows, threads_for(d, B), smem, s>>>(w, (int)d, fwht_post(d & -d), perm, signs, E, packed, row_norms);
+    if (persistent_fits(d, kBf16 ? 2 : 4)) {
+        const size_t psmem = pers_smem(d, kBf16 ? 2 : 4);
+        auto kp = quantize_persistent<B, kBf16, BITS, kSym>;
+        st = prep(kp, psmem);
+        if (st != WQ_OK) return st;
+        if (prefer_persistent(kp, psmem, k, smem, threads)) {
+            kp<<<persistent_grid(kp, threads, psmem, rows), threads, psmem, s>>>(
+                w, (int)rows, (int)d, fwht_post(d & -d), perm, signs, E, packed, row_norms);
+            return launch_status();
+        }
+    }
+    k<<<(unsigned)rows, threads, smem, s>>>(w, (int)d, fwht_post(d & -d), perm, signs, E, packed, row_norms);
     return launch_status();
 }
 
@@ -554,6 +863,13 @@ wq_status dequantize_unrotate(const uint8_t *packed, const void *row_norms, int 
         case 6: return deq_dt<6>(nb, ob, bits, packed, row_norms, rows, d, cb, perm, signs, out, s);
         default: return WQ_ERR_SHAPE;
     }
+}
+
+unsigned int read_and_clear_fault() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_fault, sizeof v) != cudaSuccess) return 0x80000000u;
+    if (v) cudaMemcpyToSymbol(g_fault, &zero, sizeof zero);
+    return v;
 }
 
 }  // namespace rpbh_fast

@@ -24,5 +24,8 @@ wq_status dequantize_unrotate(const uint8_t *packed, const void *row_norms, int 
                               int bits, const float *codebook, const int32_t *perm, const int8_t *signs, void *out,
                               int out_dtype, cudaStream_t s);
 
+// Reads and clears the fault bits of these kernels (bit 1: a bounded wait for a row copy ran out).
+unsigned int read_and_clear_fault();
+
 }  // namespace rpbh_fast
 }  // namespace wq

@@ -24,6 +24,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "rpbh_fast.cuh"
 #include "wq.h"
 
 namespace wq {
@@ -180,8 +181,9 @@ __global__ void __launch_bounds__(kThreads, 4)
         for (int b = 0; b < kBoxes; ++b)
             tma_load_2d(tile + b * kBoxBytes, &tmap, b * (kBf16In ? 64 : 32), blockIdx.x * kRows, bar);
     }
-    if (!mbar_wait_bounded(bar, 0, kMaxPolls)) {
-        if (lane == 0) atomicOr(&g_fault, 1u);
+    // the bounded wait's outcome is made CTA-uniform so that no lane is left inside a shuffle
+    if (__syncthreads_or(!mbar_wait_bounded(bar, 0, kMaxPolls))) {
+        if (threadIdx.x == 0) atomicOr(&g_fault, 1u);
         mbar_wait_bounded(bar, 0, kMaxPolls);  // give an in-flight copy a second chance to land
         return;
     }
@@ -502,6 +504,8 @@ extern "C" wq_status wq_device_fault(unsigned int *flags) {
     unsigned int v = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&v, tq3::g_fault, sizeof v) != cudaSuccess) return WQ_ERR_CUDA;
     if (v && cudaMemcpyToSymbol(tq3::g_fault, &zero, sizeof zero) != cudaSuccess) return WQ_ERR_CUDA;
-    *flags = v;
+    const unsigned int r = rpbh_fast::read_and_clear_fault();
+    if (r & 0x80000000u) return WQ_ERR_CUDA;
+    *flags = v | r;
     return WQ_OK;
 }
