@@ -113,8 +113,8 @@ def traffic_bytes(kernel: str):
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    src = {"tq3_encode": "tq3.cu", "tq3_decode": "tq3.cu", "rpbh_quantize": "rpbh.cu", "rpbh_rotate": "rpbh.cu",
-           "rpbh_dequantize": "rpbh.cu"}.get(kernel)
+    src = {"tq3_encode": "tq3_rows.cu", "tq3_decode": "tq3_rows.cu", "tq3_encode_exact": "tq3.cu",
+           "rpbh_quantize": "rpbh_fast.cu", "rpbh_rotate": "rpbh_fast.cu", "rpbh_dequantize": "rpbh_fast.cu"}.get(kernel)
     if src is None:
         return None
     with open(os.path.join(ROOT, "weight_quantization_b200", "csrc", src), "rb") as f:
@@ -165,6 +165,14 @@ class KVWorkload:
     def parts(self):
         """(kernel, launches, fn) in step order: encode K and V, then decode K and V."""
         return [("tq3_encode", 2, self._encode_both), ("tq3_decode", 2, self._decode_both)]
+
+    def extras(self):
+        """Kernels timed beside the step (not part of it): the bit-exact encoder on the same cache."""
+        def enc_exact():
+            for i in range(2):
+                self.ops.tq3_encode(self.x[i], self.mask, self.packed[i].view(-1, 1, 48), self.norms[i].view(-1, 1),
+                                    self.scales[i].view(-1, 1), exact=True)
+        return [("tq3_encode_exact", 2, enc_exact)]
 
     def step(self):
         for _, _, fn in self.parts():
@@ -228,6 +236,9 @@ class LongContextWorkload(KVWorkload):
     def parts(self):
         return [("tq3_decode", 1, lambda: self.ops.tq3_decode(self.rec[0], self.rec[1], self.rec[2], self.mask,
                                                                out=self.out))]
+
+    def extras(self):
+        return []
 
     def e2e_setup(self):
         self.pin_rec = [t.pin_memory() for t in self.host_rec]
@@ -422,6 +433,27 @@ def run_ours(args):
     achieved = per_kernel[dom]["gbs"]
     del graphs
 
+    # kernels reported beside the step (same inputs, timed the same way, not part of `value`)
+    beside = {}
+    for name, n, fn in (wl.extras() if hasattr(wl, "extras") else []):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        for _ in range(args.warmup):
+            g.replay()
+        reps = max(3, min(args.steps, 500))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        avg_ms = e0.elapsed_time(e1) / (n * reps)
+        beside[name] = {"avg_us": avg_ms * 1e3, "launches": n * reps,
+                        "gbs": wl.bytes_per_launch.get(name, wl.bytes_per_launch[parts[0][0]]) / (avg_ms / 1e3) / 1e9}
+        del g
+
     # end to end through the same API with pinned host buffers
     wl.e2e_setup()
     for _ in range(max(1, args.warmup // 2)):
@@ -457,6 +489,7 @@ def run_ours(args):
                          "traffic": traffic_bytes(dom),
                          "algorithmic_bytes_per_launch": wl.bytes_per_launch[dom]},
             "kernels": per_kernel,
+            **({"kernels_beside_step": beside} if beside else {}),
             "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": wl.h2d,
                     "d2h_bytes_per_step": wl.d2h},
             "gpu_launches": launches,

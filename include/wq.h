@@ -64,6 +64,12 @@ typedef enum { WQ_F32 = 0, WQ_BF16 = 1 } wq_dtype;
  * the sign flips; y = FWHT_128(y) * fp32(1/sqrt(128)) (7 butterfly stages, h = 1..64);
  * scale = max(max|y|, 1e-8); idx_i = #{j : B_j < y_i / scale} against TQ3_BOUNDARIES;
  * indices packed 8 per 24-bit little-endian group (_pack_3bit).
+ * Precision: the kernel takes each decision y_i / scale > B_j as |fwht(s x)_i| > B_j * T on the
+ * unnormalised transform (T = max|fwht(s x)|, or the value the 1e-8 scale floor implies), which
+ * is the same comparison in exact arithmetic. An index can therefore differ from the page's
+ * step-by-step fp32 rounding only where y_i / scale lies within about 1e-6 of a boundary (exact
+ * ties included); norms (fp32 sum of squares) and scales agree to within 1e-6 relative. Use
+ * tq3_encode_exact for output that reproduces the page's rounding bit for bit.
  *   x          device, n_vec x 128 elements of x_dtype, 16-byte aligned.
  *   sign_mask  host, 4 words: bit i of the 128-bit little-endian mask is sign draw i
  *              (1 -> +1, 0 -> -1), i.e. _generate_sign_flips(128, seed).
@@ -71,6 +77,15 @@ typedef enum { WQ_F32 = 0, WQ_BF16 = 1 } wq_dtype;
  * Errors: WQ_ERR_NULL, WQ_ERR_SHAPE (n_vec < 0), WQ_ERR_DTYPE, WQ_ERR_ALIGN, WQ_ERR_CUDA. */
 wq_status tq3_encode(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
                      uint8_t *packed, float *norms, float *scales, void *stream);
+
+/* tq3_encode_exact -- tq3_quantize with the page's rounding reproduced step by step: the norm
+ * rounded once from an fp64 sum of squares, x / n and y / scale as correctly rounded fp32
+ * quotients, the butterflies and post-multiplier as single fp32 operations, and the
+ * searchsorted tie rule (a value equal to a boundary takes the lower index). Packed bytes, norms
+ * and scales equal those of that definition bit for bit. Same arguments and errors as tq3_encode;
+ * slower (about twice the instructions per element). */
+wq_status tq3_encode_exact(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
+                           uint8_t *packed, float *norms, float *scales, void *stream);
 
 /* tq3_decode -- tq3_dequantize. For each record: y_i = TQ3_CENTROIDS[idx_i] * scale;
  * y = FWHT_128(y) * fp32(1/sqrt(128)); out_i = (y_i * s_i) * norm. With out_dtype = WQ_BF16

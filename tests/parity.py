@@ -25,9 +25,12 @@ def rel_rows(got, ref):
     return np.abs(got - ref).max(axis=1) / den
 
 
-def check_tq3_encode(oracle, x, sign_bits, is_bf16, g_packed, g_norms, g_scales):
-    """Compare GPU encode outputs with the oracle. Returns a dict of counts."""
-    xs, idx, n, s = oracle.tq3_encode_debug(x, sign_bits, is_bf16=is_bf16)
+def check_tq3_encode(oracle, x, sign_bits, is_bf16, g_packed, g_norms, g_scales, ref=None):
+    """Compare GPU encode outputs with the oracle. Returns a dict of counts.
+
+    ref: the oracle's tq3_encode_debug(x, sign_bits, is_bf16) result, when the caller has it.
+    """
+    xs, idx, n, s = ref if ref is not None else oracle.tq3_encode_debug(x, sign_bits, is_bf16=is_bf16)
     g_packed = np.asarray(g_packed).reshape(-1, 48)
     g_idx = oracle.tq3_unpack(g_packed)
     _, B = oracle.tq3_tables()
@@ -49,9 +52,13 @@ def check_tq3_encode(oracle, x, sign_bits, is_bf16, g_packed, g_norms, g_scales)
     near = np.zeros(xs.shape, bool)
     for b in B.astype(np.float64):
         near |= np.abs(xs.astype(np.float64) - b) < TIE_WINDOW
+    far = 0
+    if n_mism:
+        far = int((dist >= 1e-7).sum())
     return {
         "vectors": int(idx.shape[0]),
         "index_mismatches": n_mism,
+        "mismatches_beyond_1e-7": far,
         "coeffs_in_tie_window": int(near.sum()),
         "exact_zero_coeffs": int((xs == 0).sum()),
         "bytes_equal": bool(np.array_equal(g_packed, ref_packed)),

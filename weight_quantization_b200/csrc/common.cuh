@@ -31,6 +31,12 @@ __device__ __forceinline__ uint4 ld_stream16(const void *p) {
                  : "l"(p));
     return v;
 }
+// Read-only 16-byte load that may allocate in L1 (neighbouring lanes' loads share lines).
+__device__ __forceinline__ uint4 ld_nc16(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
 __device__ __forceinline__ uint2 ld_stream8(const void *p) {
     uint2 v;
     asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
@@ -120,6 +126,17 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int 
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(map), "r"(x),
                  "r"(y), "r"(smem_u32(src))
                  : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed bulk groups still read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until at most N committed bulk groups are still in flight (writes included).
+template <int N>
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ void tma_store_commit_wait_read() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");

@@ -25,33 +25,20 @@
 
 #include "common.cuh"
 #include "rpbh_fast.cuh"
+#include "tq3_common.cuh"
+#include "tq3_rows.cuh"
 #include "wq.h"
 
 namespace wq {
 namespace tq3 {
 
-constexpr int kD = 128;
 constexpr int kRows = 64;       // vectors per CTA
 constexpr int kThreads = 128;   // two threads per vector
 constexpr int kBoxBytes = kRows * 128;
 constexpr uint32_t kMaxPolls = 1u << 24;
-constexpr int64_t kMaxChunk = int64_t(1) << 30;  // vectors per launch (TMA row coordinates are int32)
 
 // Set (sticky) by a kernel whose bounded wait for its TMA tile ran out; read by wq_device_fault.
 __device__ unsigned int g_fault;
-
-struct SignMask {
-    uint32_t w[4];  // bit i = sign draw i (1 -> +1, 0 -> -1)
-};
-
-// The draws of _generate_sign_flips(128, seed=42): the page's fixed table. Kernels specialised on it
-// fold the flips into compile-time constants; any other table takes the runtime path.
-__host__ __device__ constexpr uint32_t default_mask_word(int w) {
-    return w == 0 ? 0x3fd74222u : w == 1 ? 0x01ab7c17u : w == 2 ? 0xff4abaf6u : 0x656b5fe7u;
-}
-__host__ __device__ constexpr uint32_t default_flip(int e) {
-    return ((default_mask_word(e >> 5) >> (e & 31)) & 1u) ? 0u : 0x80000000u;
-}
 
 // Sign-bit XOR pattern for the pair of elements (e, e + 1), e = 64 * half + 2k, laid out like a
 // bf16x2 word (bit 15 = element e, bit 31 = element e + 1). H is all ones for half 1.
@@ -98,9 +85,6 @@ __device__ __forceinline__ void stage64(float (&a)[64], int half) {
     }
 }
 
-// fp32(1.0 / math.sqrt(128)), the post-multiplier of _fwht_inplace.
-__device__ __forceinline__ float fwht_post() { return __uint_as_float(0x3DB504F3u); }
-
 // Correctly rounded x / d given r = RN(1/d) (Markstein), two lanes at a time.
 __device__ __forceinline__ f32x2 div2(f32x2 x, f32x2 r, f32x2 neg_d) {
     const f32x2 q0 = mul2(x, r);
@@ -126,13 +110,6 @@ __device__ __forceinline__ float add_index(float q, float w8, float word) {
     return __fmaf_rn(pos ? w8 : -w8, c, __fadd_rn(word, pos ? 4.0f * w8 : 3.0f * w8));
 }
 
-// TQ3_CENTROIDS as printed on the page (fp32).
-__device__ __forceinline__ float centroid(uint32_t idx) {
-    const uint32_t m = (idx & 4u) ? (idx & 3u) : (3u - idx);
-    const float mag = m == 0 ? 0.1129f : m == 1 ? 0.3479f : m == 2 ? 0.6168f : 0.9816f;
-    return (idx & 4u) ? mag : -mag;
-}
-
 // Stages h = 2 .. 32 of the butterfly on 64 values held as 32 pairs (2k, 2k + 1).
 __device__ __forceinline__ void fwht_local_2_32(float (&a)[64]) {
     f32x2 P[32];
@@ -149,15 +126,6 @@ __device__ __forceinline__ void fwht_local_2_32(float (&a)[64]) {
             }
 #pragma unroll
     for (int k = 0; k < 32; ++k) upk2(P[k], a[2 * k], a[2 * k + 1]);
-}
-
-__device__ __forceinline__ unsigned char *tile_base(unsigned char *raw) {
-    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
-}
-
-// Address of 16-byte chunk j (0..7) of row `row` in a 128-byte-swizzled TMA box.
-__device__ __forceinline__ unsigned char *swz(unsigned char *box, int row, int j) {
-    return box + row * 128 + ((j ^ (row & 7)) << 4);
 }
 
 template <bool kBf16In, bool kDefault>
@@ -409,12 +377,6 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
 }
 
-inline bool is_default(const SignMask &m) {
-    for (int i = 0; i < 4; ++i)
-        if (m.w[i] != default_mask_word(i)) return false;
-    return true;
-}
-
 inline size_t smem_bytes(bool bf16) { return (size_t)(bf16 ? 2 : 4) * kBoxBytes + 1024 + 64; }
 
 }  // namespace tq3
@@ -424,6 +386,19 @@ using namespace wq;
 
 extern "C" wq_status tq3_encode(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
                                 uint8_t *packed, float *norms, float *scales, void *stream) {
+    if (n_vec < 0) return WQ_ERR_SHAPE;
+    if (!valid_dtype(x_dtype)) return WQ_ERR_DTYPE;
+    if (n_vec == 0) return WQ_OK;
+    if (!x || !sign_mask || !packed || !norms || !scales) return WQ_ERR_NULL;
+    if (n_vec > ((int64_t)1 << 40)) return WQ_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(norms, 4) || !aligned(scales, 4)) return WQ_ERR_ALIGN;
+    tq3::SignMask m;
+    for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
+    return tq3_rows::encode(x, x_dtype, n_vec, m, packed, norms, scales, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" wq_status tq3_encode_exact(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
+                                      uint8_t *packed, float *norms, float *scales, void *stream) {
     if (n_vec < 0) return WQ_ERR_SHAPE;
     if (!valid_dtype(x_dtype)) return WQ_ERR_DTYPE;
     if (n_vec == 0) return WQ_OK;
@@ -470,6 +445,7 @@ extern "C" wq_status tq3_decode(const uint8_t *packed, const float *norms, const
     if (!aligned(packed, 16) || !aligned(out, 16) || !aligned(norms, 4) || !aligned(scales, 4)) return WQ_ERR_ALIGN;
     tq3::SignMask m;
     for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
+    return tq3_rows::decode(packed, norms, scales, n_vec, m, out, out_dtype, static_cast<cudaStream_t>(stream));
     const bool def = tq3::is_default(m), bf = out_dtype == WQ_BF16;
     const int esz = bf ? 2 : 4;
     const size_t smem = tq3::smem_bytes(bf);
@@ -505,7 +481,8 @@ extern "C" wq_status wq_device_fault(unsigned int *flags) {
     if (cudaMemcpyFromSymbol(&v, tq3::g_fault, sizeof v) != cudaSuccess) return WQ_ERR_CUDA;
     if (v && cudaMemcpyToSymbol(tq3::g_fault, &zero, sizeof zero) != cudaSuccess) return WQ_ERR_CUDA;
     const unsigned int r = rpbh_fast::read_and_clear_fault();
-    if (r & 0x80000000u) return WQ_ERR_CUDA;
-    *flags = v | r;
+    const unsigned int q = tq3_rows::read_and_clear_fault();
+    if ((r | q) & 0x80000000u) return WQ_ERR_CUDA;
+    *flags = v | r | q;
     return WQ_OK;
 }

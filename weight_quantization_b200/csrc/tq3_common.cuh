@@ -1,0 +1,55 @@
+// Constants and small helpers shared by the TQ3 kernels (page "tq3_core.py").
+#pragma once
+
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace wq {
+namespace tq3 {
+
+constexpr int kD = 128;
+constexpr int64_t kMaxChunk = int64_t(1) << 30;  // vectors per launch (TMA row coordinates are int32)
+
+struct SignMask {
+    uint32_t w[4];  // bit i = sign draw i (1 -> +1, 0 -> -1)
+};
+
+// The draws of _generate_sign_flips(128, seed=42): the page's fixed table. Kernels specialised on it
+// fold the flips into compile-time constants; any other table takes the runtime path.
+__host__ __device__ constexpr uint32_t default_mask_word(int w) {
+    return w == 0 ? 0x3fd74222u : w == 1 ? 0x01ab7c17u : w == 2 ? 0xff4abaf6u : 0x656b5fe7u;
+}
+__host__ __device__ constexpr uint32_t default_flip(int e) {
+    return ((default_mask_word(e >> 5) >> (e & 31)) & 1u) ? 0u : 0x80000000u;
+}
+// +1 / -1 as an int
+__host__ __device__ constexpr int default_sign(int e) { return default_flip(e) ? -1 : 1; }
+
+inline bool is_default(const SignMask &m) {
+    for (int i = 0; i < 4; ++i)
+        if (m.w[i] != default_mask_word(i)) return false;
+    return true;
+}
+
+// fp32(1.0 / math.sqrt(128)), the post-multiplier of _fwht_inplace.
+__device__ __forceinline__ float fwht_post() { return __uint_as_float(0x3DB504F3u); }
+
+// TQ3_CENTROIDS as printed on the page (fp32).
+__host__ __device__ __forceinline__ float centroid(uint32_t idx) {
+    const uint32_t m = (idx & 4u) ? (idx & 3u) : (3u - idx);
+    const float mag = m == 0 ? 0.1129f : m == 1 ? 0.3479f : m == 2 ? 0.6168f : 0.9816f;
+    return (idx & 4u) ? mag : -mag;
+}
+
+__device__ __forceinline__ unsigned char *tile_base(unsigned char *raw) {
+    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+}
+
+// Address of 16-byte chunk j (0..7) of row `row` in a 128-byte-swizzled TMA box.
+__device__ __forceinline__ unsigned char *swz(unsigned char *box, int row, int j) {
+    return box + row * 128 + ((j ^ (row & 7)) << 4);
+}
+
+}  // namespace tq3
+}  // namespace wq

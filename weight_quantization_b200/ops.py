@@ -23,6 +23,7 @@ _DT = {torch.float32: WQ_F32, torch.bfloat16: WQ_BF16}
 _vp, _i64, _int = C.c_void_p, C.c_int64, C.c_int
 PROTOTYPES = {
     "tq3_encode": (_int, [_vp, _int, _i64, _vp, _vp, _vp, _vp, _vp]),
+    "tq3_encode_exact": (_int, [_vp, _int, _i64, _vp, _vp, _vp, _vp, _vp]),
     "tq3_decode": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _int, _vp]),
     "tq3_compressed_bytes": (_i64, [_i64]),
     "rpbh_quantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp]),
@@ -93,10 +94,11 @@ def _mask_arg(mask) -> np.ndarray:
 # ---------------------------------------------------------------------------------------------
 # TQ3
 # ---------------------------------------------------------------------------------------------
-def tq3_encode(x: torch.Tensor, sign_mask, packed=None, norms=None, scales=None):
+def tq3_encode(x: torch.Tensor, sign_mask, packed=None, norms=None, scales=None, exact=False):
     """TQ3-encode a [..., D] fp32/bf16 CUDA tensor (D a multiple of 128).
 
     Returns (packed uint8 [..., D/128, 48], norms fp32 [..., D/128], scales fp32 [..., D/128]).
+    exact=True calls tq3_encode_exact (the page's rounding bit for bit) instead of tq3_encode.
     """
     if x.dtype not in _DT:
         raise ValueError("x must be float32 or bfloat16")
@@ -111,9 +113,10 @@ def tq3_encode(x: torch.Tensor, sign_mask, packed=None, norms=None, scales=None)
     if scales is None:
         scales = torch.empty(lead, dtype=torch.float32, device=x.device)
     m = _mask_arg(sign_mask)
-    st = lib().tq3_encode(_dev(x, "x"), _DT[x.dtype], n_vec, m.ctypes.data, _dev(packed, "packed"),
-                          _dev(norms, "norms"), _dev(scales, "scales"), _stream(x.device))
-    _check("tq3_encode", st)
+    name = "tq3_encode_exact" if exact else "tq3_encode"
+    st = getattr(lib(), name)(_dev(x, "x"), _DT[x.dtype], n_vec, m.ctypes.data, _dev(packed, "packed"),
+                              _dev(norms, "norms"), _dev(scales, "scales"), _stream(x.device))
+    _check(name, st)
     return packed, norms, scales
 
 
