@@ -131,9 +131,10 @@ def traffic_bytes(kernel: str):
 # workloads
 # ---------------------------------------------------------------------------------------------
 class KVWorkload:
-    """TQ3 encode + decode of a bf16 KV cache (K and V)."""
+    """TQ3 encode + decode of a bf16 KV cache: K and V stored as one contiguous [2, 8, 8, 4096, 128]
+    tensor, so one encode and one decode call cover all 524,288 vectors."""
 
-    name = "tq3-kv-cache-bf16-8x8x4096x128"
+    name = "tq3-kv-cache-bf16-2x8x8x4096x128"
     unit = "vectors/s"
     metric = "TQ3 encode+decode vectors/s (K and V caches, bf16)"
 
@@ -141,61 +142,55 @@ class KVWorkload:
         from weight_quantization_b200 import ops
         self.ops = ops
         k, v = inputs.kv_cache(seed=seed)
-        self.host = [torch.from_numpy(a.reshape(-1, 128).view(np.int16)).view(torch.bfloat16) for a in (k, v)]
-        self.n_half = self.host[0].shape[0]
+        kv = np.concatenate([k.reshape(-1, 128), v.reshape(-1, 128)])
+        self.host = [torch.from_numpy(kv.view(np.int16)).view(torch.bfloat16)]
+        self.n_half = self.host[0].shape[0] // 2
         self.units = 2 * self.n_half
+        n = self.units
         self.mask = ops.sign_mask_words(inputs.tq3_sign_bits())
-        self.x = [h.to(dev) for h in self.host]
-        self.packed = [torch.empty(self.n_half, 48, dtype=torch.uint8, device=dev) for _ in range(2)]
-        self.norms = [torch.empty(self.n_half, dtype=torch.float32, device=dev) for _ in range(2)]
-        self.scales = [torch.empty(self.n_half, dtype=torch.float32, device=dev) for _ in range(2)]
-        self.out = [torch.empty(self.n_half, 128, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.x = [self.host[0].to(dev)]
+        self.packed = [torch.empty(n, 48, dtype=torch.uint8, device=dev)]
+        self.norms = [torch.empty(n, dtype=torch.float32, device=dev)]
+        self.scales = [torch.empty(n, dtype=torch.float32, device=dev)]
+        self.out = [torch.empty(n, 128, dtype=torch.bfloat16, device=dev)]
         self.kernels = ["tq3_encode", "tq3_decode"]
-        self.bytes_per_launch = {"tq3_encode": 312 * self.n_half, "tq3_decode": 312 * self.n_half}
+        self.bytes_per_launch = {"tq3_encode": 312 * n, "tq3_decode": 312 * n}
 
-    def _encode_both(self):
-        for i in range(2):
-            self.ops.tq3_encode(self.x[i], self.mask, self.packed[i].view(-1, 1, 48), self.norms[i].view(-1, 1),
-                                self.scales[i].view(-1, 1))
+    def _encode(self, exact=False):
+        self.ops.tq3_encode(self.x[0], self.mask, self.packed[0].view(-1, 1, 48), self.norms[0].view(-1, 1),
+                            self.scales[0].view(-1, 1), exact=exact)
 
-    def _decode_both(self):
-        for i in range(2):
-            self.ops.tq3_decode(self.packed[i], self.norms[i], self.scales[i], self.mask, out=self.out[i])
+    def _decode(self):
+        self.ops.tq3_decode(self.packed[0], self.norms[0], self.scales[0], self.mask, out=self.out[0])
 
     def parts(self):
-        """(kernel, launches, fn) in step order: encode K and V, then decode K and V."""
-        return [("tq3_encode", 2, self._encode_both), ("tq3_decode", 2, self._decode_both)]
+        """(kernel, launches, fn) in step order: encode the cache, then decode it."""
+        return [("tq3_encode", 1, self._encode), ("tq3_decode", 1, self._decode)]
 
     def extras(self):
         """Kernels timed beside the step (not part of it): the bit-exact encoder on the same cache."""
-        def enc_exact():
-            for i in range(2):
-                self.ops.tq3_encode(self.x[i], self.mask, self.packed[i].view(-1, 1, 48), self.norms[i].view(-1, 1),
-                                    self.scales[i].view(-1, 1), exact=True)
-        return [("tq3_encode_exact", 2, enc_exact)]
+        return [("tq3_encode_exact", 1, lambda: self._encode(exact=True))]
 
     def step(self):
         for _, _, fn in self.parts():
             fn()
 
-    # end to end: pinned host K, V in; decoded K, V and the TQ3 records out
+    # end to end: pinned host cache in; decoded cache and the TQ3 records out
     def e2e_setup(self):
         self.pin_in = [h.pin_memory() for h in self.host]
         self.pin_out = [torch.empty_like(h).pin_memory() for h in self.host]
-        self.pin_packed = [torch.empty(self.n_half, 48, dtype=torch.uint8).pin_memory() for _ in range(2)]
-        self.pin_ns = [torch.empty(2, self.n_half, dtype=torch.float32).pin_memory() for _ in range(2)]
+        self.pin_packed = [torch.empty(self.units, 48, dtype=torch.uint8).pin_memory()]
+        self.pin_ns = [torch.empty(2, self.units, dtype=torch.float32).pin_memory()]
         self.h2d = sum(t.numel() * t.element_size() for t in self.pin_in)
         self.d2h = sum(t.numel() * t.element_size() for t in self.pin_out + self.pin_packed + self.pin_ns)
 
     def e2e_step(self):
-        for i in range(2):
-            self.x[i].copy_(self.pin_in[i], non_blocking=True)
+        self.x[0].copy_(self.pin_in[0], non_blocking=True)
         self.step()
-        for i in range(2):
-            self.pin_out[i].copy_(self.out[i], non_blocking=True)
-            self.pin_packed[i].copy_(self.packed[i], non_blocking=True)
-            self.pin_ns[i][0].copy_(self.norms[i], non_blocking=True)
-            self.pin_ns[i][1].copy_(self.scales[i], non_blocking=True)
+        self.pin_out[0].copy_(self.out[0], non_blocking=True)
+        self.pin_packed[0].copy_(self.packed[0], non_blocking=True)
+        self.pin_ns[0][0].copy_(self.norms[0], non_blocking=True)
+        self.pin_ns[0][1].copy_(self.scales[0], non_blocking=True)
 
     # the oracle on a bounded sample of the same cache
     def oracle_rate(self, budget_s=10.0):

@@ -176,10 +176,12 @@ wq_status wq_gaussian_lloyd_max(int bits, int iters, float *out);
  * Errors: WQ_ERR_NULL, WQ_ERR_BITS, WQ_ERR_SHAPE (d <= 0). */
 wq_status wq_rpbh_codebook(int bits, int64_t d, float *out);
 
-/* wq_device_fault -- reads and clears the library's sticky device fault bits. A TMA kernel whose
- * bounded wait for its tile transfer runs out (which does not happen in normal operation) sets
- * bit 0 and returns early, leaving its outputs unspecified. Synchronous (a device-to-host copy on
- * the legacy default stream); `flags` is host memory. Errors: WQ_ERR_NULL, WQ_ERR_CUDA. */
+/* wq_device_fault -- reads and clears the library's sticky device fault bits. A kernel whose
+ * bounded wait runs out (which does not happen in normal operation) sets a bit and returns early,
+ * leaving its outputs unspecified: bit 0 a TQ3 kernel waiting for a TMA tile, bit 1 an RPBH kernel
+ * waiting for a row copy, bit 3 the tensor-core TQ3 encoder waiting for a tile or its product.
+ * Synchronous (a device-to-host copy on the legacy default stream); `flags` is host memory.
+ * Errors: WQ_ERR_NULL, WQ_ERR_CUDA. */
 wq_status wq_device_fault(unsigned int *flags);
 
 /* wq_status_string -- a static, NUL-terminated description of a status code. */

@@ -64,6 +64,9 @@ inline bool valid_dtype(int t) { return t == WQ_F32 || t == WQ_BF16; }
 // than the current setting (tracked per kernel and device), so that later calls -- including
 // calls made while a stream is captured into a CUDA graph -- issue no attribute change.
 bool ensure_dynamic_smem(const void *kernel, size_t smem);
+// Resident CTAs per SM for (kernel, block size, dynamic smem) on the current device, queried once
+// and cached (0 if the query fails).
+int blocks_per_sm_cached(const void *kernel, int threads, size_t smem);
 inline int dtype_size(int t) { return t == WQ_F32 ? 4 : 2; }
 
 }  // namespace wq
@@ -87,10 +90,22 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-// Waits for phase `phase` of the barrier to complete, giving up after `max_iter` polls (each poll
-// may itself suspend the warp for a hardware-defined time). Returns false on timeout.
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Upper bound on any wait for a copy or a tensor-core product (2 s: orders of magnitude above a
+// real transfer, short enough that a lost completion ends the kernel promptly).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Waits for phase `phase` of the barrier to complete, giving up after `max_iter` polls or
+// kWaitLimitNs of wall-clock time, whichever comes first (a poll may itself suspend the thread for
+// a hardware-defined time, so the clock is what bounds the wait). Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t phase, uint32_t max_iter) {
     const uint32_t a = smem_u32(bar);
+    const uint64_t t0 = global_ns();
     for (uint32_t it = 0; it < max_iter; ++it) {
         uint32_t ok;
         asm volatile(
@@ -99,6 +114,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t phase,
             : "r"(a), "r"(phase)
             : "memory");
         if (ok) return true;
+        if ((it & 63) == 63 && global_ns() - t0 > kWaitLimitNs) return false;
     }
     return false;
 }

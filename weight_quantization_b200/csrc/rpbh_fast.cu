@@ -690,11 +690,7 @@ size_t pers_smem(int64_t d, int esz) { return (size_t)PLayout((int)d, esz).total
 
 bool persistent_fits(int64_t d, int esz) { return d <= 32768 && pers_smem(d, esz) + 1024 <= smem_limit(); }
 
-int blocks_per_sm(const void *k, int threads, size_t smem) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess) return 0;
-    return n;
-}
+int blocks_per_sm(const void *k, int threads, size_t smem) { return blocks_per_sm_cached(k, threads, smem); }
 
 // The persistent form pays for its resident tables with shared memory; it is taken only when that
 // costs no resident CTAs per SM against the one-row-per-CTA form (its extra smem otherwise lowers
@@ -709,9 +705,8 @@ bool prefer_persistent(KP kp, size_t pers, KR kr, size_t plain, int threads) {
 // Grid for a persistent kernel: every SM gets as many CTAs as fit, but never more CTAs than rows.
 template <typename K>
 int persistent_grid(K k, int threads, size_t smem, int64_t rows) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, threads, smem) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
+    int per_sm = blocks_per_sm_cached(reinterpret_cast<const void *>(k), threads, smem);
+    if (per_sm < 1) per_sm = 1;
     const int64_t g = (int64_t)per_sm * sm_count();
     return (int)(g < rows ? g : rows);
 }

@@ -59,4 +59,19 @@ bool ensure_dynamic_smem(const void *kernel, size_t smem) {
     return true;
 }
 
+int blocks_per_sm_cached(const void *kernel, int threads, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::pair<std::pair<const void *, int>, std::pair<int, size_t>>, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    const auto key = std::make_pair(std::make_pair(kernel, dev), std::make_pair(threads, smem));
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess) return 0;
+    cache[key] = n;
+    return n;
+}
+
 }  // namespace wq

@@ -26,6 +26,7 @@
 #include "common.cuh"
 #include "rpbh_fast.cuh"
 #include "tq3_common.cuh"
+#include "tq3_mma.cuh"
 #include "tq3_rows.cuh"
 #include "wq.h"
 
@@ -394,7 +395,9 @@ extern "C" wq_status tq3_encode(const void *x, int x_dtype, int64_t n_vec, const
     if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(norms, 4) || !aligned(scales, 4)) return WQ_ERR_ALIGN;
     tq3::SignMask m;
     for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
-    return tq3_rows::encode(x, x_dtype, n_vec, m, packed, norms, scales, static_cast<cudaStream_t>(stream));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (x_dtype == WQ_BF16) return tq3_mma::encode_bf16(x, n_vec, m, packed, norms, scales, s);
+    return tq3_rows::encode(x, x_dtype, n_vec, m, packed, norms, scales, s);
 }
 
 extern "C" wq_status tq3_encode_exact(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
@@ -482,7 +485,8 @@ extern "C" wq_status wq_device_fault(unsigned int *flags) {
     if (v && cudaMemcpyToSymbol(tq3::g_fault, &zero, sizeof zero) != cudaSuccess) return WQ_ERR_CUDA;
     const unsigned int r = rpbh_fast::read_and_clear_fault();
     const unsigned int q = tq3_rows::read_and_clear_fault();
-    if ((r | q) & 0x80000000u) return WQ_ERR_CUDA;
-    *flags = v | r | q;
+    const unsigned int t = tq3_mma::read_and_clear_fault();
+    if ((r | q | t) & 0x80000000u) return WQ_ERR_CUDA;
+    *flags = v | r | q | t;
     return WQ_OK;
 }

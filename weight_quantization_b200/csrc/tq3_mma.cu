@@ -1,0 +1,445 @@
+// TQ3 encoder for bf16 input on sm_100a with the sign flips and the Walsh-Hadamard transform as
+// one tensor-core product: page "tq3_core.py" (tq3_quantize, _fwht_inplace, _quantize_to_indices,
+// _pack_3bit).
+//
+// For a tile of 128 vectors X[128 x 128] (bf16, loaded by TMA with 128-byte swizzling) the kernel
+// computes Z = X B^T with B[j][i] = -H[j][i] s_i, H the 128-point Hadamard matrix ((-1)^popc(i&j))
+// and s the sign flips: z_j = -fwht(s x)_j. Every product is exact (a bf16 value times +-1) and
+// the sums accumulate in fp32 in tensor memory; one tcgen05.mma per 16 columns of K, issued by a
+// single thread, eight per tile. Thread t of the CTA then owns vector t: it reads row t of the
+// accumulator (tcgen05.ld, its warp's 32-lane quarter) into 128 registers and runs the same
+// decision and packing as the CUDA-core fast encoder (norm from ||z||^2 / 128, absmax T, the
+// index as 3.5 + sgn(-z) (c + 1/2) with c = #{k : |z| > edge_k T}, 8^j-weighted fp32 words).
+// The negation in B makes an exact zero come out as z = +0, i.e. a true -0, whose index is 3 as
+// the page's searchsorted gives for 0.
+//
+// Numerics: the fp32 accumulation order of the tensor core is not the butterfly's, so z agrees
+// with the step-by-step transform to a few units in the last place relative to max|z|; as for the
+// CUDA-core fast encoder, an index can differ from the page's rounding only for a coefficient
+// within about 1e-6 of a boundary. Norms and scales agree to within 1e-6 relative.
+//
+// Pipeline per CTA (persistent over tiles): TMA load of the next tile is issued as soon as the
+// tensor core has consumed the current one, so it lands while the 128 threads run the epilogue;
+// the accumulator is read out before the next product overwrites it. Every wait is bounded: on a
+// timeout the fault flag is set, the CTA gives in-flight copies and products a bounded chance to
+// land, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "tq3_common.cuh"
+#include "tq3_mma.cuh"
+
+namespace wq {
+namespace tq3_mma {
+
+using tq3::SignMask;
+
+// A CTA holding tensor memory runs alone on its SM, so one CTA carries four independent groups of
+// 128 threads; each group streams its own tiles through its own operand buffer and accumulator
+// (128 columns each of the 512 allocated) and synchronises on its own named barrier. The epilogue
+// reads the accumulator in 32-column pieces (twice: norm and absmax, then the indices), so a
+// thread holds 32 values rather than 128 and four groups fit the register file.
+constexpr int kTile = 128;  // vectors per tile = threads per group = rows of the product
+constexpr int kGroups = 4;
+constexpr int kThreads = kGroups * kTile;
+constexpr int kBox = kTile * 128;  // one 64-column half of a 128 x 128 bf16 operand (128 B per row)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kMaxPolls = 1u << 24;
+// shared-memory layout (offsets from a 1024-byte aligned base): B, then one A per group, then per
+// group its full (TMA) and done (tensor core) barriers, then the TMEM address
+constexpr int kStageBytes = 2 * kBox;
+constexpr int kOffB = 0;
+constexpr int kOffA = 2 * kBox;
+constexpr int kOffBar = kOffA + kGroups * kStageBytes;
+constexpr int kSmem = 1024 + kOffBar + 32 * kGroups + 16;  // ... TMEM address, then the B barrier
+
+// Plain barrier over the 128 threads of group g.
+__device__ __forceinline__ void group_sync(int g) { asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory"); }
+
+// __syncthreads_or over the 128 threads of group g (named barrier 1 + g).
+__device__ __forceinline__ bool group_sync_or(int g, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(1 + g)
+        : "memory");
+    return r != 0;
+}
+
+__device__ unsigned int g_fault;
+
+// ---------------------------------------------------------------------------------------------
+// tcgen05 wrappers (sm_100a PTX)
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A * B^T, both operands K-major bf16 in shared memory, fp32 accumulator.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// The barrier receives one arrival once every tensor-core operation this thread issued is done.
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major operand stored with the 128-byte swizzle: rows of
+// 128 bytes, 8-row atoms 1024 bytes apart (stride byte offset), leading byte offset unused (1),
+// descriptor version 1, layout type 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, N = 128, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+// 32 consecutive accumulator columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3]), "=f"(r[4]), "=f"(r[5]), "=f"(r[6]), "=f"(r[7]),
+          "=f"(r[8]), "=f"(r[9]), "=f"(r[10]), "=f"(r[11]), "=f"(r[12]), "=f"(r[13]), "=f"(r[14]), "=f"(r[15]),
+          "=f"(r[16]), "=f"(r[17]), "=f"(r[18]), "=f"(r[19]), "=f"(r[20]), "=f"(r[21]), "=f"(r[22]), "=f"(r[23]),
+          "=f"(r[24]), "=f"(r[25]), "=f"(r[26]), "=f"(r[27]), "=f"(r[28]), "=f"(r[29]), "=f"(r[30]), "=f"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// The positive TQ3_BOUNDARIES (fp32).
+__device__ __forceinline__ float edge(int k) { return k == 0 ? 0.2304f : k == 1 ? 0.4824f : 0.7992f; }
+
+// Chunks c0 .. c0 + 3 of row n of B = -H diag(s), K-major with the 128-byte swizzle (two 64-column
+// halves): entry (n, k) is -(-1)^popc(n & k) s_k, exactly +-1 in bf16.
+template <bool kFold>
+__device__ __forceinline__ void build_b(unsigned char *B, const SignMask &mask, int n, int c0) {
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {  // 16-byte chunk c holds k = 8c .. 8c + 7
+        const int c = c0 + cc;
+        uint32_t w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            uint32_t pair = 0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int k = 8 * c + 2 * u + h;
+                const uint32_t sneg = kFold ? ((~tq3::default_mask_word(k >> 5) >> (k & 31)) & 1u)
+                                            : ((~mask.w[k >> 5] >> (k & 31)) & 1u);
+                const uint32_t neg = ((uint32_t)__popc(n & k) & 1u) ^ sneg ^ 1u;
+                pair |= (neg ? 0xBF80u : 0x3F80u) << (16 * h);
+            }
+            w[u] = pair;
+        }
+        unsigned char *half = B + (c >> 3) * kBox;
+        *reinterpret_cast<uint4 *>(half + n * 128 + (((c & 7) ^ (n & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// B for the page's sign table, built at compile time in the shared-memory layout above (8192
+// words), so that a CTA fetches it with one bulk copy instead of computing it.
+struct BTable {
+    uint32_t w[2 * kBox / 4];
+};
+constexpr int popc_parity(int v) {
+    int p = 0;
+    for (; v; v &= v - 1) p ^= 1;
+    return p;
+}
+constexpr BTable make_default_b() {
+    BTable t{};
+    for (int n = 0; n < kTile; ++n)
+        for (int c = 0; c < 16; ++c)
+            for (int u = 0; u < 4; ++u) {
+                uint32_t pair = 0;
+                for (int h = 0; h < 2; ++h) {
+                    const int k = 8 * c + 2 * u + h;
+                    const uint32_t sneg = (~tq3::default_mask_word(k >> 5) >> (k & 31)) & 1u;
+                    const uint32_t neg = (uint32_t)popc_parity(n & k) ^ sneg ^ 1u;
+                    pair |= (neg ? 0xBF80u : 0x3F80u) << (16 * h);
+                }
+                const int byte = (c >> 3) * kBox + n * 128 + (((c & 7) ^ (n & 7)) << 4) + 4 * u;
+                t.w[byte / 4] = pair;
+            }
+    return t;
+}
+__device__ __align__(128) const BTable kDefaultB = make_default_b();
+
+template <bool kFold>
+__global__ void __launch_bounds__(kThreads, 1)
+    encode_mma(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, SignMask mask, uint8_t *__restrict__ packed,
+               float *__restrict__ norms, float *__restrict__ scales) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *const base = tq3::tile_base(smem_raw);
+    const int grp = threadIdx.x >> 7, tid = threadIdx.x & 127, warp = tid >> 5;
+    unsigned char *const B = base + kOffB;
+    unsigned char *const A = base + kOffA + grp * kStageBytes;
+    uint64_t *const full = reinterpret_cast<uint64_t *>(base + kOffBar) + 4 * grp;
+    uint64_t *const done = full + 1;
+    uint32_t *const tslot = reinterpret_cast<uint32_t *>(base + kOffBar + 32 * kGroups);
+    uint64_t *const bready = reinterpret_cast<uint64_t *>(base + kOffBar + 32 * kGroups + 8);
+    const int64_t n_tiles = (n_vec + kTile - 1) / kTile;
+    // streams interleave across CTAs (stream = grp * gridDim.x + blockIdx.x), so the tiles left
+    // over after whole rounds spread one per SM rather than piling onto the first CTAs
+    const int64_t stream = (int64_t)grp * gridDim.x + blockIdx.x, n_streams = (int64_t)gridDim.x * kGroups;
+    const int64_t my_tiles = stream < n_tiles ? (n_tiles - stream + n_streams - 1) / n_streams : 0;
+
+    if (!kFold) {
+        build_b<kFold>(B, mask, threadIdx.x >> 2, 4 * (threadIdx.x & 3));
+        fence_proxy_async_smem();  // B is written by threads and read by the tensor core
+    }
+    if (tid == 0) {
+        mbar_init(full, 1);
+        mbar_init(done, 1);
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bready, 1);
+        if (kFold) {
+            mbar_expect_tx(bready, 2 * kBox);
+            bulk_load(B, &kDefaultB, 2 * kBox, bready);
+        } else {
+            mbar_expect_tx(bready, 0);  // completes the phase at once: B was written above
+        }
+    }
+    if (threadIdx.x < 32) tmem_alloc(tslot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot + (uint32_t)(grp * kTile);  // this group's 128 columns
+    const uint32_t my_lanes = tmem + ((uint32_t)(warp * 32) << 16);
+
+    // Thread 0 of the group drives the pipeline: the load of tile i + 1 is issued once the product
+    // of tile i has consumed the operand buffer (it lands during tile i's epilogue), and the
+    // product of tile i + 1 once every thread has finished reading tile i's accumulator.
+    int64_t n_loaded = 0, n_landed = 0, n_mma = 0;  // thread 0's counters (for the fault path)
+    auto issue_load = [&](int64_t i) {
+        const int y = (int)((stream + i * n_streams) * kTile);
+        mbar_expect_tx(full, kStageBytes);
+        tma_load_2d(A, &tmap, 0, y, full);
+        tma_load_2d(A + kBox, &tmap, 64, y, full);
+        n_loaded = i + 1;
+    };
+    const uint64_t adesc = sw128_desc(smem_u32(A)), bdesc = sw128_desc(smem_u32(B));
+    auto issue_mma = [&](int64_t i) -> bool {
+        if (i == 0 && !mbar_wait_bounded(bready, 0u, kMaxPolls)) return false;
+        if (!mbar_wait_bounded(full, (uint32_t)(i & 1), kMaxPolls)) return false;
+        n_landed = i + 1;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {  // K = 16 per instruction: 32 bytes into a 128-byte row
+            const uint32_t off = (uint32_t)((ks >> 2) * kBox + (ks & 3) * 32) >> 4;
+            mma_bf16(tmem, adesc + off, bdesc + off, kIdesc, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(done);
+        n_mma = i + 1;
+        return true;
+    };
+    bool next_ok = true;  // thread 0: the product of the coming tile was issued
+    if (tid == 0 && my_tiles > 0) {
+        issue_load(0);
+        next_ok = issue_mma(0);
+    }
+
+    const float post = tq3::fwht_post();
+    bool fault = false;
+    int64_t n_done = 0;
+    for (int64_t it = 0; it < my_tiles; ++it) {
+        bool ok = next_ok;
+        if (tid == 0 && ok) ok = mbar_wait_bounded(done, (uint32_t)(it & 1), kMaxPolls);
+        if (group_sync_or(grp, !ok)) {
+            fault = true;
+            break;
+        }
+        n_done = it + 1;
+        // the product has consumed the operand buffer: the next tile lands during this epilogue
+        if (tid == 0 && it + 1 < my_tiles) issue_load(it + 1);
+        tc_fence_after();
+
+        // pass 1: ||x||^2 = ||z||^2 / 128 (Parseval) and max|z|
+        f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
+        float mm[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            float z[32];
+            tmem_ld32(my_lanes + 32 * c, z);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const f32x2 p = pk2(z[2 * i], z[2 * i + 1]);
+                acc[i & 3] = fma2(p, p, acc[i & 3]);
+                mm[i & 3] = max3(mm[i & 3], fabsf(z[2 * i]), fabsf(z[2 * i + 1]));
+            }
+        }
+        float n2;
+        {
+            float a0, a1;
+            upk2(add2(add2(acc[0], acc[1]), add2(acc[2], acc[3])), a0, a1);
+            n2 = __fadd_rn(a0, a1);
+        }
+        const float m = fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3]));
+        float nrm0 = __fsqrt_rn(__fmul_rn(n2, 0.0078125f));
+        // the fp32 squares overflowed: sum them in fp64 (taken by the whole warp, since the
+        // accumulator reads are warp-collective; lanes that do not need it discard the result)
+        const bool big = !(n2 <= 3.0e38f);
+        if (__any_sync(0xffffffffu, big)) {
+            double d = 0.0;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float z[32];
+                tmem_ld32(my_lanes + 32 * c, z);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) d = __fma_rn((double)z[i], (double)z[i], d);
+            }
+            if (big) nrm0 = __double2float_rn(__dsqrt_rn(d * 0.0078125));
+        }
+        const float nrm = fmaxf(nrm0, 1e-8f);
+        const float sraw = __fmul_rn(__fdiv_rn(m, nrm), post);
+        const float scale = fmaxf(sraw, 1e-8f);
+        const float T = (sraw >= 1e-8f) ? m : __fmul_rn(__fmul_rn(1e-8f, nrm), 11.3137085f);
+        const float t0 = __fmul_rn(edge(0), T), t1 = __fmul_rn(edge(1), T), t2 = __fmul_rn(edge(2), T);
+        const uint32_t Mb = (277u - ((__float_as_uint(t0) >> 23) & 0xffu)) << 23;  // 1 / ulp(t0)
+        const float M = __uint_as_float(Mb);
+        const float K0 = -__fmul_rn(t0, M), K1 = -__fmul_rn(t1, M), K2 = -__fmul_rn(t2, M);
+
+        // pass 2, 32 columns (groups 4c .. 4c + 3) at a time. Group q (elements 8q .. 8q + 7) is
+        // accumulated as two fp32 words, even slots and odd slots, each starting from
+        // sum_j 3.5 * 8^j over its slots; slot 0 (even) is added first, so every later partial
+        // sum is an integer below 2^24.
+        const int64_t v = (stream + it * n_streams) * kTile + tid;
+        uint8_t *const rec = packed + v * 48;
+        const f32x2 HALF = pk2(0.5f, 0.5f);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            float z[32];
+            tmem_ld32(my_lanes + 32 * c, z);
+            tmem_ld_wait();
+            f32x2 W[4];
+#pragma unroll
+            for (int gg = 0; gg < 4; ++gg) W[gg] = pk2(932067.5f, 7456540.0f);
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int gg = 0; gg < 4; ++gg) {
+                    const int i = 4 * gg + p;  // local elements 2i (slot 2p) and 2i + 1 (slot 2p + 1)
+                    const float za = z[2 * i], zb = z[2 * i + 1];
+                    const uint32_t wa = 0x80000000u | ((127u + 6u * p) << 23);      // -8^(2p)
+                    const uint32_t wb = 0x80000000u | ((127u + 6u * p + 3u) << 23);  // -8^(2p+1)
+                    const uint32_t ha = __float_as_uint(za) & 0x80000000u, hb = __float_as_uint(zb) & 0x80000000u;
+                    const float sMa = __uint_as_float(ha | Mb), sMb = __uint_as_float(hb | Mb);
+                    const f32x2 w2 = pk2(__uint_as_float(ha ^ wa), __uint_as_float(hb ^ wb));
+                    // c + 1/2 from the three exact 0/1 steps, then one fused update of the word
+                    const f32x2 s0 = pk2(__saturatef(__fmaf_rn(za, sMa, K0)), __saturatef(__fmaf_rn(zb, sMb, K0)));
+                    const f32x2 s1 = pk2(__saturatef(__fmaf_rn(za, sMa, K1)), __saturatef(__fmaf_rn(zb, sMb, K1)));
+                    const f32x2 s2 = pk2(__saturatef(__fmaf_rn(za, sMa, K2)), __saturatef(__fmaf_rn(zb, sMb, K2)));
+                    W[gg] = fma2(w2, add2(add2(s0, s1), add2(s2, HALF)), W[gg]);
+                }
+            if (c == 3) {
+                // the accumulator has been read: the next product may overwrite it
+                tc_fence_before();
+                group_sync(grp);
+                if (tid == 0 && it + 1 < my_tiles) next_ok = issue_mma(it + 1);
+            }
+            uint32_t g4[4];
+#pragma unroll
+            for (int gg = 0; gg < 4; ++gg) {
+                float lo, hi;
+                upk2(W[gg], lo, hi);
+                g4[gg] = __float2uint_rn(__fadd_rn(lo, hi));
+            }
+            if (v < n_vec) {  // _pack_3bit: groups 4c .. 4c + 3 are bytes 12c .. 12c + 11, little-endian
+                uint32_t *o = reinterpret_cast<uint32_t *>(rec + 12 * c);
+                o[0] = g4[0] | (g4[1] << 24);
+                o[1] = (g4[1] >> 8) | (g4[2] << 16);
+                o[2] = (g4[2] >> 16) | (g4[3] << 8);
+            }
+        }
+        if (v < n_vec) {
+            norms[v] = nrm;
+            scales[v] = scale;
+        }
+    }
+    if (fault && tid == 0) {
+        atomicOr(&g_fault, 8u);
+        // give what is still in flight a bounded chance to land before the memory goes away
+        for (int64_t i = n_landed; i < n_loaded; ++i) mbar_wait_bounded(full, (uint32_t)(i & 1), kMaxPolls);
+        if (n_mma > n_done) mbar_wait_bounded(done, (uint32_t)(n_done & 1), kMaxPolls);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        tc_fence_after();
+        tmem_dealloc(*tslot, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------------
+namespace {
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (!cached[dev]) cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev);
+    return cached[dev];
+}
+
+template <typename K>
+wq_status launch(K k, int64_t cnt, const CUtensorMap &tm, const SignMask &m, uint8_t *pc, float *nc, float *sc,
+                 cudaStream_t s) {
+    if (!ensure_dynamic_smem(reinterpret_cast<const void *>(k), kSmem)) return WQ_ERR_CUDA;
+    // one CTA per SM (it holds all 512 tensor-memory columns), never more CTAs than tile triples
+    const int64_t tiles = (cnt + kTile - 1) / kTile;
+    const int64_t triples = (tiles + kGroups - 1) / kGroups;
+    const int64_t g_ = sm_count() > 0 ? sm_count() : 1;
+    const int64_t g = g_ < triples ? g_ : triples;
+    k<<<(unsigned)g, kThreads, kSmem, s>>>(cnt, tm, m, pc, nc, sc);
+    return launch_status();
+}
+}  // namespace
+
+wq_status encode_bf16(const void *x, int64_t n_vec, const SignMask &m, uint8_t *packed, float *norms, float *scales,
+                      cudaStream_t s) {
+    const bool def = tq3::is_default(m);
+    for (int64_t off = 0; off < n_vec; off += tq3::kMaxChunk) {
+        const int64_t cnt = n_vec - off < tq3::kMaxChunk ? n_vec - off : tq3::kMaxChunk;
+        const unsigned char *xc = static_cast<const unsigned char *>(x) + off * (tq3::kD * 2);
+        CUtensorMap tm;
+        if (!make_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xc, tq3::kD, (uint64_t)cnt, tq3::kD * 2, 64, kTile))
+            return WQ_ERR_CUDA;
+        const wq_status st = def ? launch(encode_mma<true>, cnt, tm, m, packed + off * 48, norms + off, scales + off, s)
+                                 : launch(encode_mma<false>, cnt, tm, m, packed + off * 48, norms + off, scales + off, s);
+        if (st != WQ_OK) return st;
+    }
+    return WQ_OK;
+}
+
+unsigned int read_and_clear_fault() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_fault, sizeof v) != cudaSuccess) return 0x80000000u;
+    if (v) cudaMemcpyToSymbol(g_fault, &zero, sizeof zero);
+    return v;
+}
+
+}  // namespace tq3_mma
+}  // namespace wq

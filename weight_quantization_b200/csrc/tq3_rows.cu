@@ -489,9 +489,8 @@ int sm_count() {
 // Persistent grid: as many CTAs as fit on the GPU at once, never more than there are tiles.
 template <typename K>
 int grid_for(K k, size_t smem, int64_t tiles) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, kThreads, smem) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
+    int per_sm = blocks_per_sm_cached(reinterpret_cast<const void *>(k), kThreads, smem);
+    if (per_sm < 1) per_sm = 1;
     const int64_t g = (int64_t)per_sm * (sm_count() > 0 ? sm_count() : 1);
     return (int)(g < tiles ? g : tiles);
 }
