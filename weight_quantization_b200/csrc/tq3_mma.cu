@@ -124,7 +124,27 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&r)[32]) {
         : "r"(taddr)
         : "memory");
 }
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Waits for this thread's outstanding accumulator reads. The registers of the read being waited for
+// pass through the statement, so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_wait(float (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+f"(r[0]), "+f"(r[1]), "+f"(r[2]), "+f"(r[3]), "+f"(r[4]), "+f"(r[5]), "+f"(r[6]), "+f"(r[7]),
+                   "+f"(r[8]), "+f"(r[9]), "+f"(r[10]), "+f"(r[11]), "+f"(r[12]), "+f"(r[13]), "+f"(r[14]), "+f"(r[15]),
+                   "+f"(r[16]), "+f"(r[17]), "+f"(r[18]), "+f"(r[19]), "+f"(r[20]), "+f"(r[21]), "+f"(r[22]), "+f"(r[23]),
+                   "+f"(r[24]), "+f"(r[25]), "+f"(r[26]), "+f"(r[27]), "+f"(r[28]), "+f"(r[29]), "+f"(r[30]), "+f"(r[31])
+                 :
+                 : "memory");
+}
+
+// Sum of squares (two lanes at a time) and absmax of a 32-column piece.
+__device__ __forceinline__ void acc_piece(const float (&z)[32], f32x2 (&acc)[4], float (&mm)[4]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const f32x2 p = pk2(z[2 * i], z[2 * i + 1]);
+        acc[i & 3] = fma2(p, p, acc[i & 3]);
+        mm[i & 3] = max3(mm[i & 3], fabsf(z[2 * i]), fabsf(z[2 * i + 1]));
+    }
+}
 
 // The positive TQ3_BOUNDARIES (fp32).
 __device__ __forceinline__ float edge(int k) { return k == 0 ? 0.2304f : k == 1 ? 0.4824f : 0.7992f; }
@@ -152,6 +172,49 @@ __device__ __forceinline__ void build_b(unsigned char *B, const SignMask &mask, 
         }
         unsigned char *half = B + (c >> 3) * kBox;
         *reinterpret_cast<uint4 *>(half + n * 128 + (((c & 7) ^ (n & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// Indices of one 32-column piece (elements 32c .. 32c + 31, groups 4c .. 4c + 3) packed into the
+// record's bytes 12c .. 12c + 11 (_pack_3bit: group i is bytes 3i .. 3i + 2, little-endian).
+// Group q is accumulated as two fp32 words, even slots and odd slots, each starting from
+// sum_j 3.5 * 8^j over its slots; each step adds +-8^j (c + 1/2), an integer except for slot 0
+// (+-1/2), which comes first, so every partial sum is an integer below 2^24 and the words are exact.
+__device__ __forceinline__ void bucket_piece(const float (&z)[32], uint32_t Mb, float K0, float K1, float K2,
+                                             uint8_t *rec, int c, bool store) {
+    const f32x2 HALF = pk2(0.5f, 0.5f);
+    f32x2 W[4];
+#pragma unroll
+    for (int gg = 0; gg < 4; ++gg) W[gg] = pk2(932067.5f, 7456540.0f);
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+        for (int gg = 0; gg < 4; ++gg) {
+            const int i = 4 * gg + p;  // local elements 2i (slot 2p) and 2i + 1 (slot 2p + 1)
+            const float za = z[2 * i], zb = z[2 * i + 1];
+            const uint32_t wa = 0x80000000u | ((127u + 6u * p) << 23);      // -8^(2p)
+            const uint32_t wb = 0x80000000u | ((127u + 6u * p + 3u) << 23);  // -8^(2p+1)
+            const uint32_t ha = __float_as_uint(za) & 0x80000000u, hb = __float_as_uint(zb) & 0x80000000u;
+            const float sMa = __uint_as_float(ha | Mb), sMb = __uint_as_float(hb | Mb);
+            const f32x2 w2 = pk2(__uint_as_float(ha ^ wa), __uint_as_float(hb ^ wb));
+            // c + 1/2 from the three exact 0/1 steps, then one fused update of the word
+            const f32x2 s0 = pk2(__saturatef(__fmaf_rn(za, sMa, K0)), __saturatef(__fmaf_rn(zb, sMb, K0)));
+            const f32x2 s1 = pk2(__saturatef(__fmaf_rn(za, sMa, K1)), __saturatef(__fmaf_rn(zb, sMb, K1)));
+            const f32x2 s2 = pk2(__saturatef(__fmaf_rn(za, sMa, K2)), __saturatef(__fmaf_rn(zb, sMb, K2)));
+            W[gg] = fma2(w2, add2(add2(s0, s1), add2(s2, HALF)), W[gg]);
+        }
+    uint32_t g4[4];
+#pragma unroll
+    for (int gg = 0; gg < 4; ++gg) {
+        float lo, hi;
+        upk2(W[gg], lo, hi);
+        g4[gg] = __float2uint_rn(__fadd_rn(lo, hi));
+    }
+    if (store) {
+        uint32_t *o = reinterpret_cast<uint32_t *>(rec + 12 * c);
+        o[0] = g4[0] | (g4[1] << 24);
+        o[1] = (g4[1] >> 8) | (g4[2] << 16);
+        o[2] = (g4[2] >> 16) | (g4[3] << 8);
     }
 }
 
@@ -281,13 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 4; ++c) {
             float z[32];
             tmem_ld32(my_lanes + 32 * c, z);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const f32x2 p = pk2(z[2 * i], z[2 * i + 1]);
-                acc[i & 3] = fma2(p, p, acc[i & 3]);
-                mm[i & 3] = max3(mm[i & 3], fabsf(z[2 * i]), fabsf(z[2 * i + 1]));
-            }
+            tmem_wait(z);
+            acc_piece(z, acc, mm);
         }
         float n2;
         {
@@ -306,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 4; ++c) {
                 float z[32];
                 tmem_ld32(my_lanes + 32 * c, z);
-                tmem_ld_wait();
+                tmem_wait(z);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) d = __fma_rn((double)z[i], (double)z[i], d);
             }
@@ -321,58 +379,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float M = __uint_as_float(Mb);
         const float K0 = -__fmul_rn(t0, M), K1 = -__fmul_rn(t1, M), K2 = -__fmul_rn(t2, M);
 
-        // pass 2, 32 columns (groups 4c .. 4c + 3) at a time. Group q (elements 8q .. 8q + 7) is
-        // accumulated as two fp32 words, even slots and odd slots, each starting from
-        // sum_j 3.5 * 8^j over its slots; slot 0 (even) is added first, so every later partial
-        // sum is an integer below 2^24.
+        // pass 2: the indices, 32 columns at a time
         const int64_t v = (stream + it * n_streams) * kTile + tid;
         uint8_t *const rec = packed + v * 48;
-        const f32x2 HALF = pk2(0.5f, 0.5f);
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            float z[32];
-            tmem_ld32(my_lanes + 32 * c, z);
-            tmem_ld_wait();
-            f32x2 W[4];
-#pragma unroll
-            for (int gg = 0; gg < 4; ++gg) W[gg] = pk2(932067.5f, 7456540.0f);
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-#pragma unroll
-                for (int gg = 0; gg < 4; ++gg) {
-                    const int i = 4 * gg + p;  // local elements 2i (slot 2p) and 2i + 1 (slot 2p + 1)
-                    const float za = z[2 * i], zb = z[2 * i + 1];
-                    const uint32_t wa = 0x80000000u | ((127u + 6u * p) << 23);      // -8^(2p)
-                    const uint32_t wb = 0x80000000u | ((127u + 6u * p + 3u) << 23);  // -8^(2p+1)
-                    const uint32_t ha = __float_as_uint(za) & 0x80000000u, hb = __float_as_uint(zb) & 0x80000000u;
-                    const float sMa = __uint_as_float(ha | Mb), sMb = __uint_as_float(hb | Mb);
-                    const f32x2 w2 = pk2(__uint_as_float(ha ^ wa), __uint_as_float(hb ^ wb));
-                    // c + 1/2 from the three exact 0/1 steps, then one fused update of the word
-                    const f32x2 s0 = pk2(__saturatef(__fmaf_rn(za, sMa, K0)), __saturatef(__fmaf_rn(zb, sMb, K0)));
-                    const f32x2 s1 = pk2(__saturatef(__fmaf_rn(za, sMa, K1)), __saturatef(__fmaf_rn(zb, sMb, K1)));
-                    const f32x2 s2 = pk2(__saturatef(__fmaf_rn(za, sMa, K2)), __saturatef(__fmaf_rn(zb, sMb, K2)));
-                    W[gg] = fma2(w2, add2(add2(s0, s1), add2(s2, HALF)), W[gg]);
-                }
-            if (c == 3) {
-                // the accumulator has been read: the next product may overwrite it
-                tc_fence_before();
-                group_sync(grp);
-                if (tid == 0 && it + 1 < my_tiles) next_ok = issue_mma(it + 1);
-            }
-            uint32_t g4[4];
-#pragma unroll
-            for (int gg = 0; gg < 4; ++gg) {
-                float lo, hi;
-                upk2(W[gg], lo, hi);
-                g4[gg] = __float2uint_rn(__fadd_rn(lo, hi));
-            }
-            if (v < n_vec) {  // _pack_3bit: groups 4c .. 4c + 3 are bytes 12c .. 12c + 11, little-endian
-                uint32_t *o = reinterpret_cast<uint32_t *>(rec + 12 * c);
-                o[0] = g4[0] | (g4[1] << 24);
-                o[1] = (g4[1] >> 8) | (g4[2] << 16);
-                o[2] = (g4[2] >> 16) | (g4[3] << 8);
-            }
-        }
+        const bool store = v < n_vec;
+        // the pieces alternate between two register sets, so each piece's read from tensor
+        // memory overlaps the previous piece's work
+        float za[32], zb[32];
+        tmem_ld32(my_lanes + 0, za);
+        tmem_wait(za);
+        tmem_ld32(my_lanes + 32, zb);
+        bucket_piece(za, Mb, K0, K1, K2, rec, 0, store);
+        tmem_wait(zb);
+        tmem_ld32(my_lanes + 64, za);
+        bucket_piece(zb, Mb, K0, K1, K2, rec, 1, store);
+        tmem_wait(za);
+        tmem_ld32(my_lanes + 96, zb);
+        bucket_piece(za, Mb, K0, K1, K2, rec, 2, store);
+        tmem_wait(zb);
+        // the accumulator has been read: the next product runs during the last piece's work
+        tc_fence_before();
+        group_sync(grp);
+        if (tid == 0 && it + 1 < my_tiles) next_ok = issue_mma(it + 1);
+        bucket_piece(zb, Mb, K0, K1, K2, rec, 3, store);
         if (v < n_vec) {
             norms[v] = nrm;
             scales[v] = scale;
