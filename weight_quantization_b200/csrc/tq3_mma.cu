@@ -38,7 +38,7 @@ using tq3::SignMask;
 
 // A CTA holding tensor memory runs alone on its SM, so one CTA carries four independent groups of
 // 128 threads; each group streams its own tiles through its own operand buffer and accumulator
-// (128 columns each of the 512 allocated) and synchronises on its own named barrier. The epilogue
+// (128 columns each of the 512 allocated), coordinated by mbarriers only. The epilogue
 // reads the accumulator in 32-column pieces (twice: norm and absmax, then the indices), so a
 // thread holds 32 values rather than 128 and four groups fit the register file.
 constexpr int kTile = 128;  // vectors per tile = threads per group = rows of the product
@@ -55,20 +55,6 @@ constexpr int kOffA = 2 * kBox;
 constexpr int kOffBar = kOffA + kGroups * kStageBytes;
 constexpr int kSmem = 1024 + kOffBar + 32 * kGroups + 16;  // ... TMEM address, then the B barrier
 
-// Plain barrier over the 128 threads of group g.
-__device__ __forceinline__ void group_sync(int g) { asm volatile("bar.sync %0, 128;" ::"r"(1 + g) : "memory"); }
-
-// __syncthreads_or over the 128 threads of group g (named barrier 1 + g).
-__device__ __forceinline__ bool group_sync_or(int g, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, 128, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(1 + g)
-        : "memory");
-    return r != 0;
-}
 
 __device__ unsigned int g_fault;
 
@@ -258,6 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char *const A = base + kOffA + grp * kStageBytes;
     uint64_t *const full = reinterpret_cast<uint64_t *>(base + kOffBar) + 4 * grp;
     uint64_t *const done = full + 1;
+    uint64_t *const empty = full + 2;  // one arrival per warp once it has read the accumulator
     uint32_t *const tslot = reinterpret_cast<uint32_t *>(base + kOffBar + 32 * kGroups);
     uint64_t *const bready = reinterpret_cast<uint64_t *>(base + kOffBar + 32 * kGroups + 8);
     const int64_t n_tiles = (n_vec + kTile - 1) / kTile;
@@ -273,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         mbar_init(full, 1);
         mbar_init(done, 1);
+        mbar_init(empty, kTile / 32);
     }
     if (threadIdx.x == 0) {
         mbar_init(bready, 1);
@@ -325,10 +313,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float post = tq3::fwht_post();
     bool fault = false;
     int64_t n_done = 0;
+    // No thread waits for the others in this loop: every thread waits on the product's barrier
+    // itself, each warp reports on `empty` when it has read the accumulator, and only thread 0
+    // waits for those reports before it issues the next product. A timeout ends the warp's loop
+    // (the decision is warp-uniform, as the accumulator reads are warp-collective).
     for (int64_t it = 0; it < my_tiles; ++it) {
-        bool ok = next_ok;
-        if (tid == 0 && ok) ok = mbar_wait_bounded(done, (uint32_t)(it & 1), kMaxPolls);
-        if (group_sync_or(grp, !ok)) {
+        bool ok = mbar_wait_bounded(done, (uint32_t)(it & 1), kMaxPolls);
+        if (tid == 0) ok = ok && next_ok;
+        if (!__all_sync(0xffffffffu, ok)) {
             fault = true;
             break;
         }
@@ -399,8 +391,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait(zb);
         // the accumulator has been read: the next product runs during the last piece's work
         tc_fence_before();
-        group_sync(grp);
-        if (tid == 0 && it + 1 < my_tiles) next_ok = issue_mma(it + 1);
+        __syncwarp();
+        if ((tid & 31) == 0) mbar_arrive(empty);
+        if (tid == 0 && it + 1 < my_tiles)
+            next_ok = mbar_wait_bounded(empty, (uint32_t)(it & 1), kMaxPolls) && issue_mma(it + 1);
         bucket_piece(zb, Mb, K0, K1, K2, rec, 3, store);
         if (v < n_vec) {
             norms[v] = nrm;
