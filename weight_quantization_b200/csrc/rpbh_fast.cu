@@ -228,6 +228,43 @@ __device__ __forceinline__ uint32_t bucketize(float u, const Edges &E) {
     }
 }
 
+// pack_codes for one group of 32 codes (code i in byte i of cw): BITS 32-bit words of the MSB-first
+// stream, word k holding stream bits 32k .. 32k + 31 with the first at bit 31. Code i occupies
+// stream bits BITS*i .. BITS*i + BITS - 1; one that crosses a word boundary is split between two.
+template <int BITS>
+__device__ __forceinline__ void pack32(const uint32_t (&cw)[8], uint32_t (&word)[BITS]) {
+#pragma unroll
+    for (int k = 0; k < BITS; ++k) word[k] = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const uint32_t c = __byte_perm(cw[i >> 2], 0u, 0x4440u + (uint32_t)(i & 3));
+        const int o = BITS * i, k = o >> 5, r = o & 31;
+        if (r + BITS <= 32) {
+            word[k] += c << (32 - r - BITS);
+        } else {
+            word[k] += c >> (r + BITS - 32);
+            word[k + 1] += c << (64 - r - BITS);
+        }
+    }
+}
+// unpack_codes for one group: the inverse of pack32, code i into byte i of cw.
+template <int BITS>
+__device__ __forceinline__ void unpack32(const uint32_t (&word)[BITS], uint32_t (&cw)[8]) {
+    constexpr uint32_t kMask = (1u << BITS) - 1u;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) cw[q] = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int o = BITS * i, k = o >> 5, r = o & 31;
+        uint32_t c;
+        if (r + BITS <= 32)
+            c = (word[k] >> (32 - r - BITS)) & kMask;
+        else
+            c = ((word[k] << (r + BITS - 32)) | (word[k + 1] >> (64 - r - BITS))) & kMask;
+        cw[i >> 2] += c << (8 * (i & 3));
+    }
+}
+
 template <int B, bool kBf16, int BITS, bool kSym>
 __global__ void __launch_bounds__(kMaxThreads)
     quantize_kernel(const void *__restrict__ w, int d, float post, const int32_t *__restrict__ perm,
@@ -288,14 +325,10 @@ __global__ void __launch_bounds__(kMaxThreads)
         const uint4 c0 = *reinterpret_cast<const uint4 *>(raw + 32 * g);
         const uint4 c1 = *reinterpret_cast<const uint4 *>(raw + 32 * g + 16);
         const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-        unsigned __int128 acc = 0;
+        uint32_t word[BITS];
+        pack32<BITS>(cw, word);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc = (acc << BITS) | ((cw[i >> 2] >> (8 * (i & 3))) & 0xffu);
-#pragma unroll
-        for (int k = 0; k < BITS; ++k) {
-            const uint32_t word = (uint32_t)(acc >> (32 * (BITS - 1 - k)));
-            reinterpret_cast<uint32_t *>(dst + 4 * BITS * g)[k] = __byte_perm(word, 0, 0x0123);
-        }
+        for (int k = 0; k < BITS; ++k) reinterpret_cast<uint32_t *>(dst + 4 * BITS * g)[k] = __byte_perm(word[k], 0, 0x0123);
     }
     if (threadIdx.x == 0) {
         if (kBf16)
@@ -331,21 +364,12 @@ __global__ void __launch_bounds__(kMaxThreads)
     // unpack_codes: BITS big-endian words -> 32 codes
     const uint8_t *src = packed + (row * (int64_t)d / 8) * BITS;
     for (int g = threadIdx.x; g < d / 32; g += blockDim.x) {
-        unsigned __int128 acc = 0;
+        uint32_t word[BITS];
 #pragma unroll
         for (int k = 0; k < BITS; ++k)
-            acc = (acc << 32) | __byte_perm(__ldg(reinterpret_cast<const uint32_t *>(src + 4 * BITS * g) + k), 0, 0x0123);
+            word[k] = __byte_perm(__ldg(reinterpret_cast<const uint32_t *>(src + 4 * BITS * g) + k), 0, 0x0123);
         uint32_t cw[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            uint32_t wv = 0;
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int i = 4 * q + b;
-                wv |= (uint32_t)((acc >> (BITS * (31 - i))) & ((1u << BITS) - 1)) << (8 * b);
-            }
-            cw[q] = wv;
-        }
+        unpack32<BITS>(word, cw);
         *reinterpret_cast<uint4 *>(codes + 32 * g) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         *reinterpret_cast<uint4 *>(codes + 32 * g + 16) = make_uint4(cw[4], cw[5], cw[6], cw[7]);
     }
@@ -400,30 +424,10 @@ struct PLayout {
         row0 = bits + a16(d / 8);
         row1 = row0 + d * esz;
         buf = row1 + d * esz;
-        bar = buf + 4 * d;
-        total = bar + 16;
+        bar = buf + 4 * d;  // row barriers 0 and 1, table barrier 2
+        total = bar + 32;
     }
 };
-
-// Tables into shared memory: perm as 16-bit indices (clamped into the row), signs as bits
-// (bit t of word w set when signs[32 w + t] is negative).
-__device__ __forceinline__ void load_tables(uint16_t *perm16, uint32_t *sbits, const int32_t *__restrict__ perm,
-                                            const int8_t *__restrict__ signs, int d) {
-    for (int j = threadIdx.x; j < d; j += blockDim.x) perm16[j] = (uint16_t)clampi(__ldg(perm + j), d);
-    for (int w = threadIdx.x; w < d / 32; w += blockDim.x) {
-        uint32_t bits = 0;
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-            const int4 v = __ldg(reinterpret_cast<const int4 *>(signs + 32 * w) + q);
-            const uint32_t wv[4] = {(uint32_t)v.x, (uint32_t)v.y, (uint32_t)v.z, (uint32_t)v.w};
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int b = 0; b < 4; ++b) bits |= ((wv[u] >> (8 * b + 7)) & 1u) << (16 * q + 4 * u + b);
-        }
-        sbits[w] = bits;
-    }
-}
 
 // pass 0 from the staged row: y[t] = x[perm[j0 + t]] * signs[j0 + t] (the sign as a bit flip)
 template <int B, bool kBf16>
@@ -459,6 +463,55 @@ __device__ __forceinline__ bool row_ready(uint64_t *bar, uint32_t parity) {
     return !any_fail;
 }
 
+// Prologue of the persistent kernels. The tables arrive by bulk copy into buffers the row loop
+// reuses later (perm as int32 into the transpose buffer, signs into the second row buffer), and
+// the CTA's first row into the first row buffer; the tables are then converted in place: perm to
+// 16-bit indices clamped into the row, signs to bits (bit t of word w set when signs[32 w + t] is
+// negative). Returns false, CTA-uniformly and with the fault flag set, if the tables never land.
+__device__ bool persistent_prologue(const PLayout &Lo, unsigned char *base, const int32_t *__restrict__ perm,
+                                    const int8_t *__restrict__ signs, int d, const unsigned char *first_row,
+                                    uint32_t row_bytes) {
+    uint16_t *perm16 = reinterpret_cast<uint16_t *>(base + Lo.perm);
+    uint32_t *sbits = reinterpret_cast<uint32_t *>(base + Lo.bits);
+    unsigned char *rb0 = base + Lo.row0, *rb1 = base + Lo.row1, *buf = base + Lo.buf;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + Lo.bar);
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        mbar_init(&bar[2], 1);
+        mbar_expect_tx(&bar[2], 5u * (uint32_t)d);
+        bulk_load(buf, perm, 4u * (uint32_t)d, &bar[2]);
+        bulk_load(rb1, signs, (uint32_t)d, &bar[2]);
+        if (first_row) {
+            mbar_expect_tx(&bar[0], row_bytes);
+            bulk_load(rb0, first_row, row_bytes, &bar[0]);
+        }
+    }
+    __syncthreads();  // the barriers are initialised before anyone waits on them
+    if (!row_ready(&bar[2], 0)) {
+        if (threadIdx.x == 0 && first_row) mbar_wait_bounded(&bar[0], 0, kMaxPolls);
+        return false;
+    }
+    const int32_t *p32 = reinterpret_cast<const int32_t *>(buf);
+    for (int j = threadIdx.x; j < d; j += blockDim.x) perm16[j] = (uint16_t)clampi(p32[j], d);
+    for (int w = threadIdx.x; w < d / 32; w += blockDim.x) {
+        uint32_t bits = 0;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(rb1 + 32 * w + 16 * q);
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) bits |= ((wv[u] >> (8 * b + 7)) & 1u) << (16 * q + 4 * u + b);
+        }
+        sbits[w] = bits;
+    }
+    fence_proxy_async_smem();  // these reads of buf and rb1 precede the bulk copies that reuse them
+    __syncthreads();
+    return true;
+}
+
 template <int B, bool kBf16>
 __global__ void __launch_bounds__(kMaxThreads)
     rotate_persistent(const void *__restrict__ x, int rows, int d, float post, const int32_t *__restrict__ perm,
@@ -474,18 +527,11 @@ __global__ void __launch_bounds__(kMaxThreads)
     unsigned char *buf = base + Lo.buf;
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + Lo.bar);
     const uint32_t row_bytes = (uint32_t)d * esz;
-    load_tables(perm16, sbits, perm, signs, d);
-    if (threadIdx.x == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
-    }
-    __syncthreads();
     const unsigned char *xb = static_cast<const unsigned char *>(x);
     int row = blockIdx.x;
-    if (threadIdx.x == 0 && row < rows) {
-        mbar_expect_tx(&bar[0], row_bytes);
-        bulk_load(rb0, xb + (int64_t)row * row_bytes, row_bytes, &bar[0]);
-    }
+    if (!persistent_prologue(Lo, base, perm, signs, d, row < rows ? xb + (int64_t)row * row_bytes : nullptr,
+                             row_bytes))
+        return;
     const int nslots = d >> B;
     for (int it = 0; row < rows; ++it, row += gridDim.x) {
         const int cur = it & 1;
@@ -545,18 +591,11 @@ __global__ void __launch_bounds__(kMaxThreads)
     float *fb = reinterpret_cast<float *>(buf);
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + Lo.bar);
     const uint32_t row_bytes = (uint32_t)d * esz;
-    load_tables(perm16, sbits, perm, signs, d);
-    if (threadIdx.x == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
-    }
-    __syncthreads();
     const unsigned char *wb = static_cast<const unsigned char *>(w);
     int row = blockIdx.x;
-    if (threadIdx.x == 0 && row < rows) {
-        mbar_expect_tx(&bar[0], row_bytes);
-        bulk_load(rb0, wb + (int64_t)row * row_bytes, row_bytes, &bar[0]);
-    }
+    if (!persistent_prologue(Lo, base, perm, signs, d, row < rows ? wb + (int64_t)row * row_bytes : nullptr,
+                             row_bytes))
+        return;
     const int nslots = d >> B;
     for (int it = 0; row < rows; ++it, row += gridDim.x) {
         const int cur = it & 1;
@@ -609,14 +648,11 @@ __global__ void __launch_bounds__(kMaxThreads)
             const uint4 c0 = *reinterpret_cast<const uint4 *>((rb0 + cur * row_bytes) + 32 * g);
             const uint4 c1 = *reinterpret_cast<const uint4 *>((rb0 + cur * row_bytes) + 32 * g + 16);
             const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-            unsigned __int128 acc = 0;
+            uint32_t word[BITS];
+            pack32<BITS>(cw, word);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc = (acc << BITS) | ((cw[i >> 2] >> (8 * (i & 3))) & 0xffu);
-#pragma unroll
-            for (int k = 0; k < BITS; ++k) {
-                const uint32_t word = (uint32_t)(acc >> (32 * (BITS - 1 - k)));
-                reinterpret_cast<uint32_t *>(dst + 4 * BITS * g)[k] = __byte_perm(word, 0, 0x0123);
-            }
+            for (int k = 0; k < BITS; ++k)
+                reinterpret_cast<uint32_t *>(dst + 4 * BITS * g)[k] = __byte_perm(word[k], 0, 0x0123);
         }
         if (threadIdx.x == 0) {
             if (kBf16)
@@ -692,14 +728,14 @@ bool persistent_fits(int64_t d, int esz) { return d <= 32768 && pers_smem(d, esz
 
 int blocks_per_sm(const void *k, int threads, size_t smem) { return blocks_per_sm_cached(k, threads, smem); }
 
-// The persistent form pays for its resident tables with shared memory; it is taken only when that
-// costs no resident CTAs per SM against the one-row-per-CTA form (its extra smem otherwise lowers
-// the number of rows in flight, which is what keeps HBM busy here).
+// The persistent form (tables resident, rows double-buffered by bulk copies) is taken whenever it
+// fits on an SM: measured faster than one row per CTA for the LLM and DiT shapes even where its
+// larger shared-memory footprint leaves fewer CTAs per SM.
 template <typename KP, typename KR>
 bool prefer_persistent(KP kp, size_t pers, KR kr, size_t plain, int threads) {
-    const int a = blocks_per_sm(reinterpret_cast<const void *>(kp), threads, pers);
-    const int b = blocks_per_sm(reinterpret_cast<const void *>(kr), threads, plain);
-    return a >= 1 && a >= b;
+    (void)kr;
+    (void)plain;
+    return blocks_per_sm(reinterpret_cast<const void *>(kp), threads, pers) >= 1;
 }
 
 // Grid for a persistent kernel: every SM gets as many CTAs as fit, but never more CTAs than rows.
