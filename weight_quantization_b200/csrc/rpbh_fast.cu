@@ -574,7 +574,7 @@ __global__ void __launch_bounds__(kMaxThreads)
 }
 
 template <int B, bool kBf16, int BITS, bool kSym>
-__global__ void __launch_bounds__(kMaxThreads)
+__global__ void __launch_bounds__(kMaxThreads, 2)
     quantize_persistent(const void *__restrict__ w, int rows, int d, float post, const int32_t *__restrict__ perm,
                         const int8_t *__restrict__ signs, Edges E, uint8_t *__restrict__ packed,
                         void *__restrict__ row_norms) {
@@ -588,7 +588,6 @@ __global__ void __launch_bounds__(kMaxThreads)
     uint32_t *sbits = reinterpret_cast<uint32_t *>(base + Lo.bits);
     unsigned char *const rb0 = base + Lo.row0;  // row buffers rb0 and rb0 + row_bytes
     unsigned char *buf = base + Lo.buf;
-    float *fb = reinterpret_cast<float *>(buf);
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + Lo.bar);
     const uint32_t row_bytes = (uint32_t)d * esz;
     const unsigned char *wb = static_cast<const unsigned char *>(w);
@@ -615,31 +614,42 @@ __global__ void __launch_bounds__(kMaxThreads)
             store_row<B>(buf, y, blk, r);
         }
         __syncthreads();
+        // pass 1 keeps w_rot in registers (the host guarantees nslots <= kSlots * blockDim.x):
+        // thread slots s = threadIdx.x + k blockDim.x, k < kSlots, in the order of the plain loop
+        constexpr int kSlots = 64 / G::S;
+        float zk[kSlots][G::S];
         double ss = 0.0;
-        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
-            const int blk = s >> B, c = s & (G::S - 1);
-            float y[G::S];
-            load_col<B>(y, buf, blk, c);
-            butterfly<G::S>(y);
 #pragma unroll
-            for (int t = 0; t < G::S; ++t) {
-                const float z = __fmul_rn(y[t], post);
-                fb[bufpos<B>(blk, t, c)] = z;
-                const double dz = (double)z;
-                ss = __fma_rn(dz, dz, ss);
+        for (int k = 0; k < kSlots; ++k) {
+            const int s = threadIdx.x + k * (int)blockDim.x;
+            if (s < nslots) {
+                const int blk = s >> B, c = s & (G::S - 1);
+                load_col<B>(zk[k], buf, blk, c);
+                butterfly<G::S>(zk[k]);
+#pragma unroll
+                for (int t = 0; t < G::S; ++t) {
+                    zk[k][t] = __fmul_rn(zk[k][t], post);
+                    const double dz = (double)zk[k][t];
+                    ss = __fma_rn(dz, dz, ss);
+                }
             }
         }
         const float rho = __double2float_rn(__dsqrt_rn(block_sum_f64(ss, red)));
         const float den = __fadd_rn(rho, 1e-10f);
         const float rden = __frcp_rn(den);
-        for (int s = threadIdx.x; s < nslots; s += blockDim.x) {
-            const int blk = s >> B, c = s & (G::S - 1);
 #pragma unroll
-            for (int t = 0; t < G::S; ++t) {
-                const float z = fb[bufpos<B>(blk, t, c)];
-                const float q0 = __fmul_rn(z, rden);
-                const float u = __fmaf_rn(__fmaf_rn(-q0, den, z), rden, q0);
-                (rb0 + cur * row_bytes)[blk * G::H + c + (t << B)] = (uint8_t)bucketize<BITS, kSym>(u, E);
+        for (int k = 0; k < kSlots; ++k) {
+            const int s = threadIdx.x + k * (int)blockDim.x;
+            if (s < nslots) {
+                const int blk = s >> B, c = s & (G::S - 1);
+                unsigned char *cb = (rb0 + cur * row_bytes) + blk * G::H + c;
+#pragma unroll
+                for (int t = 0; t < G::S; ++t) {
+                    const float z = zk[k][t];
+                    const float q0 = __fmul_rn(z, rden);
+                    const float u = __fmaf_rn(__fmaf_rn(-q0, den, z), rden, q0);
+                    cb[t << B] = (uint8_t)bucketize<BITS, kSym>(u, E);
+                }
             }
         }
         __syncthreads();
@@ -790,7 +800,8 @@ wq_status quantize_b(const void *w, int64_t rows, int64_t d, const int32_t *perm
     auto k = quantize_kernel<B, kBf16, BITS, kSym>;
     wq_status st = prep(k, smem);
     if (st != WQ_OK) return st;
-    if (persistent_fits(d, kBf16 ? 2 : 4)) {
+    // the persistent form keeps each thread's slots of the row in registers: at most 64 / S of them
+    if (persistent_fits(d, kBf16 ? 2 : 4) && (d >> B) <= (int64_t)(64 >> B) * threads) {
         const size_t psmem = pers_smem(d, kBf16 ? 2 : 4);
         auto kp = quantize_persistent<B, kBf16, BITS, kSym>;
         st = prep(kp, psmem);
