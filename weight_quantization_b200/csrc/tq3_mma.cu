@@ -132,6 +132,18 @@ __device__ __forceinline__ void acc_piece(const float (&z)[32], f32x2 (&acc)[4],
     }
 }
 
+// (a & b) | c and (a & b) ^ c as single three-input logic operations.
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ uint32_t lop3_and_xor(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
 // The positive TQ3_BOUNDARIES (fp32).
 __device__ __forceinline__ float edge(int k) { return k == 0 ? 0.2304f : k == 1 ? 0.4824f : 0.7992f; }
 
@@ -180,9 +192,11 @@ __device__ __forceinline__ void bucket_piece(const float (&z)[32], uint32_t Mb, 
             const float za = z[2 * i], zb = z[2 * i + 1];
             const uint32_t wa = 0x80000000u | ((127u + 6u * p) << 23);      // -8^(2p)
             const uint32_t wb = 0x80000000u | ((127u + 6u * p + 3u) << 23);  // -8^(2p+1)
-            const uint32_t ha = __float_as_uint(za) & 0x80000000u, hb = __float_as_uint(zb) & 0x80000000u;
-            const float sMa = __uint_as_float(ha | Mb), sMb = __uint_as_float(hb | Mb);
-            const f32x2 w2 = pk2(__uint_as_float(ha ^ wa), __uint_as_float(hb ^ wb));
+            // copysign(M, z) and copysign(8^j, -z), one three-input logic operation each
+            const float sMa = __uint_as_float(lop3_and_or(__float_as_uint(za), 0x80000000u, Mb));
+            const float sMb = __uint_as_float(lop3_and_or(__float_as_uint(zb), 0x80000000u, Mb));
+            const f32x2 w2 = pk2(__uint_as_float(lop3_and_xor(__float_as_uint(za), 0x80000000u, wa)),
+                                 __uint_as_float(lop3_and_xor(__float_as_uint(zb), 0x80000000u, wb)));
             // c + 1/2 from the three exact 0/1 steps, then one fused update of the word
             const f32x2 s0 = pk2(__saturatef(__fmaf_rn(za, sMa, K0)), __saturatef(__fmaf_rn(zb, sMb, K0)));
             const f32x2 s1 = pk2(__saturatef(__fmaf_rn(za, sMa, K1)), __saturatef(__fmaf_rn(zb, sMb, K1)));
@@ -318,7 +332,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // waits for those reports before it issues the next product. A timeout ends the warp's loop
     // (the decision is warp-uniform, as the accumulator reads are warp-collective).
     for (int64_t it = 0; it < my_tiles; ++it) {
-        bool ok = mbar_wait_bounded(done, (uint32_t)(it & 1), kMaxPolls);
+        // one lane per warp polls the product's barrier; the warp synchronises on its answer
+        bool ok = true;
+        if ((tid & 31) == 0) ok = mbar_wait_bounded(done, (uint32_t)(it & 1), kMaxPolls);
         if (tid == 0) ok = ok && next_ok;
         if (!__all_sync(0xffffffffu, ok)) {
             fault = true;
