@@ -132,6 +132,14 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
                  : "memory");
 }
 
+// 1-D bulk copy shared -> global of `bytes` (multiple of 16, both addresses 16-byte aligned), in the
+// current bulk group (commit with bulk_commit, wait with bulk_wait_read / bulk_wait_all).
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+                 "r"(bytes)
+                 : "memory");
+}
+
 // 2-D tiled bulk load global -> shared, completing on `bar` (no multicast).
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
     asm volatile(

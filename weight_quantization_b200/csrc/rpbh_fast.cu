@@ -537,6 +537,7 @@ __global__ void __launch_bounds__(kMaxThreads)
         const int cur = it & 1;
         const int nrow = row + gridDim.x;
         if (threadIdx.x == 0 && nrow < rows) {
+            bulk_wait_read<0>();  // the store of the row that last used the other buffer has read it
             mbar_expect_tx(&bar[cur ^ 1], row_bytes);
             bulk_load((rb0 + (cur ^ 1) * row_bytes), xb + (int64_t)nrow * row_bytes, row_bytes, &bar[cur ^ 1]);
         }
@@ -566,11 +567,15 @@ __global__ void __launch_bounds__(kMaxThreads)
                     reinterpret_cast<float *>((rb0 + cur * row_bytes))[j] = z;
             }
         }
+        // the rotated row goes out with one bulk copy; the buffer is refilled only once it has been read
+        fence_proxy_async_smem();
         __syncthreads();
-        copy_out(static_cast<unsigned char *>(out) + (int64_t)row * row_bytes, (rb0 + cur * row_bytes), row_bytes);
-        fence_proxy_async_smem();  // these generic accesses precede the bulk copy that reuses (rb0 + cur * row_bytes)
-        __syncthreads();
+        if (threadIdx.x == 0) {
+            bulk_store(static_cast<unsigned char *>(out) + (int64_t)row * row_bytes, rb0 + cur * row_bytes, row_bytes);
+            bulk_commit();
+        }
     }
+    if (threadIdx.x == 0) bulk_wait_all<0>();
 }
 
 template <int B, bool kBf16, int BITS, bool kSym>
