@@ -155,6 +155,20 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int 
                  "r"(y), "r"(smem_u32(src))
                  : "memory");
 }
+// L2 policy that makes the lines it tags the first candidates for eviction (written data then goes
+// back to HBM during the kernel that produced it rather than during the next one).
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// 2-D tiled bulk store shared -> global with an L2 cache policy.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap *map, int x, int y, const void *src, uint64_t pol) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(
+                     map),
+                 "r"(x), "r"(y), "r"(smem_u32(src)), "l"(pol)
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N committed bulk groups still read their shared-memory source.
 template <int N>

@@ -465,9 +465,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
+            // decoded output is written once and read by a later kernel: evict it from L2 first
+            const uint64_t pol = l2_evict_first_policy();
 #pragma unroll
             for (int b = 0; b < G::kBoxes; ++b)
-                tma_store_2d(&omap, b * (kBf16Out ? 64 : 32), (int)(tile * kTile), buf + b * kBoxBytes);
+                tma_store_2d_hint(&omap, b * (kBf16Out ? 64 : 32), (int)(tile * kTile), buf + b * kBoxBytes, pol);
             bulk_commit();
         }
         cur = nxt;
