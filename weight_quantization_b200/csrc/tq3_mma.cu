@@ -132,6 +132,13 @@ __device__ __forceinline__ void acc_piece(const float (&z)[32], f32x2 (&acc)[4],
     }
 }
 
+// atomicAdd on shared memory with acquire-release ordering (CTA scope); returns the old value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+    return old;
+}
+
 // (a & b) | c and (a & b) ^ c as single three-input logic operations.
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
@@ -173,13 +180,14 @@ __device__ __forceinline__ void build_b(unsigned char *B, const SignMask &mask, 
     }
 }
 
-// Indices of one 32-column piece (elements 32c .. 32c + 31, groups 4c .. 4c + 3) packed into the
-// record's bytes 12c .. 12c + 11 (_pack_3bit: group i is bytes 3i .. 3i + 2, little-endian).
+// Indices of one 32-column piece (elements 32c .. 32c + 31, groups 4c .. 4c + 3) packed as the
+// record's bytes 12c .. 12c + 11, three little-endian words (_pack_3bit: group i is bytes
+// 3i .. 3i + 2).
 // Group q is accumulated as two fp32 words, even slots and odd slots, each starting from
 // sum_j 3.5 * 8^j over its slots; each step adds +-8^j (c + 1/2), an integer except for slot 0
 // (+-1/2), which comes first, so every partial sum is an integer below 2^24 and the words are exact.
 __device__ __forceinline__ void bucket_piece(const float (&z)[32], uint32_t Mb, float K0, float K1, float K2,
-                                             uint8_t *rec, int c, bool store) {
+                                             uint32_t &o0, uint32_t &o1, uint32_t &o2) {
     const f32x2 HALF = pk2(0.5f, 0.5f);
     f32x2 W[4];
 #pragma unroll
@@ -210,12 +218,9 @@ __device__ __forceinline__ void bucket_piece(const float (&z)[32], uint32_t Mb, 
         upk2(W[gg], lo, hi);
         g4[gg] = __float2uint_rn(__fadd_rn(lo, hi));
     }
-    if (store) {
-        uint32_t *o = reinterpret_cast<uint32_t *>(rec + 12 * c);
-        o[0] = g4[0] | (g4[1] << 24);
-        o[1] = (g4[1] >> 8) | (g4[2] << 16);
-        o[2] = (g4[2] >> 16) | (g4[3] << 8);
-    }
+    o0 = g4[0] | (g4[1] << 24);
+    o1 = (g4[1] >> 8) | (g4[2] << 16);
+    o2 = (g4[2] >> 16) | (g4[3] << 8);
 }
 
 // B for the page's sign table, built at compile time in the shared-memory layout above (8192
@@ -258,7 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char *const A = base + kOffA + grp * kStageBytes;
     uint64_t *const full = reinterpret_cast<uint64_t *>(base + kOffBar) + 4 * grp;
     uint64_t *const done = full + 1;
-    uint64_t *const empty = full + 2;  // one arrival per warp once it has read the accumulator
+    // per-group counters: warps that have finished reading the accumulator (modulo 4), products issued
+    uint32_t *const readers = reinterpret_cast<uint32_t *>(full + 2);
+    uint32_t *const issued = readers + 1;
     uint32_t *const tslot = reinterpret_cast<uint32_t *>(base + kOffBar + 32 * kGroups);
     uint64_t *const bready = reinterpret_cast<uint64_t *>(base + kOffBar + 32 * kGroups + 8);
     const int64_t n_tiles = (n_vec + kTile - 1) / kTile;
@@ -274,7 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         mbar_init(full, 1);
         mbar_init(done, 1);
-        mbar_init(empty, kTile / 32);
+        *readers = 0;
+        *issued = 0;
     }
     if (threadIdx.x == 0) {
         mbar_init(bready, 1);
@@ -292,10 +300,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tslot + (uint32_t)(grp * kTile);  // this group's 128 columns
     const uint32_t my_lanes = tmem + ((uint32_t)(warp * 32) << 16);
 
-    // Thread 0 of the group drives the pipeline: the load of tile i + 1 is issued once the product
-    // of tile i has consumed the operand buffer (it lands during tile i's epilogue), and the
-    // product of tile i + 1 once every thread has finished reading tile i's accumulator.
-    int64_t n_loaded = 0, n_landed = 0, n_mma = 0;  // thread 0's counters (for the fault path)
+    // Thread 0 of the group issues the loads: tile i + 1 once the product of tile i has consumed the
+    // operand buffer (it lands during tile i's epilogue). The product of tile i + 1 is issued by
+    // whichever warp is the last to finish reading tile i's accumulator, so no warp waits for the
+    // others.
+    int64_t n_loaded = 0;  // thread 0's count of loads issued (for the fault path)
     auto issue_load = [&](int64_t i) {
         const int y = (int)((stream + i * n_streams) * kTile);
         mbar_expect_tx(full, kStageBytes);
@@ -304,10 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         n_loaded = i + 1;
     };
     const uint64_t adesc = sw128_desc(smem_u32(A)), bdesc = sw128_desc(smem_u32(B));
-    auto issue_mma = [&](int64_t i) -> bool {
-        if (i == 0 && !mbar_wait_bounded(bready, 0u, kMaxPolls)) return false;
-        if (!mbar_wait_bounded(full, (uint32_t)(i & 1), kMaxPolls)) return false;
-        n_landed = i + 1;
+    auto issue_mma = [&](int64_t i) {
+        if (i == 0 && !mbar_wait_bounded(bready, 0u, kMaxPolls)) return;
+        if (!mbar_wait_bounded(full, (uint32_t)(i & 1), kMaxPolls)) return;  // the product's waiters time out
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {  // K = 16 per instruction: 32 bytes into a 128-byte row
@@ -315,32 +323,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_bf16(tmem, adesc + off, bdesc + off, kIdesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(done);
-        n_mma = i + 1;
-        return true;
+        *issued = (uint32_t)(i + 1);
     };
-    bool next_ok = true;  // thread 0: the product of the coming tile was issued
     if (tid == 0 && my_tiles > 0) {
         issue_load(0);
-        next_ok = issue_mma(0);
+        issue_mma(0);
     }
 
     const float post = tq3::fwht_post();
     bool fault = false;
-    int64_t n_done = 0;
-    // No thread waits for the others in this loop: every thread waits on the product's barrier
-    // itself, each warp reports on `empty` when it has read the accumulator, and only thread 0
-    // waits for those reports before it issues the next product. A timeout ends the warp's loop
-    // (the decision is warp-uniform, as the accumulator reads are warp-collective).
+    // No warp waits for another in this loop: each waits on the product's barrier itself, and the
+    // last warp to finish reading the accumulator issues the next product. A timeout ends the
+    // warp's loop (the decision is warp-uniform, as the accumulator reads are warp-collective).
     for (int64_t it = 0; it < my_tiles; ++it) {
         // one lane per warp polls the product's barrier; the warp synchronises on its answer
         bool ok = true;
         if ((tid & 31) == 0) ok = mbar_wait_bounded(done, (uint32_t)(it & 1), kMaxPolls);
-        if (tid == 0) ok = ok && next_ok;
         if (!__all_sync(0xffffffffu, ok)) {
             fault = true;
             break;
         }
-        n_done = it + 1;
         // the product has consumed the operand buffer: the next tile lands during this epilogue
         if (tid == 0 && it + 1 < my_tiles) issue_load(it + 1);
         tc_fence_after();
@@ -390,40 +392,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         // pass 2: the indices, 32 columns at a time
         const int64_t v = (stream + it * n_streams) * kTile + tid;
         uint8_t *const rec = packed + v * 48;
-        const bool store = v < n_vec;
+        uint32_t o[12];
         // the pieces alternate between two register sets, so each piece's read from tensor
         // memory overlaps the previous piece's work
         float za[32], zb[32];
         tmem_ld32(my_lanes + 0, za);
         tmem_wait(za);
         tmem_ld32(my_lanes + 32, zb);
-        bucket_piece(za, Mb, K0, K1, K2, rec, 0, store);
+        bucket_piece(za, Mb, K0, K1, K2, o[0], o[1], o[2]);
         tmem_wait(zb);
         tmem_ld32(my_lanes + 64, za);
-        bucket_piece(zb, Mb, K0, K1, K2, rec, 1, store);
+        bucket_piece(zb, Mb, K0, K1, K2, o[3], o[4], o[5]);
         tmem_wait(za);
         tmem_ld32(my_lanes + 96, zb);
-        bucket_piece(za, Mb, K0, K1, K2, rec, 2, store);
+        bucket_piece(za, Mb, K0, K1, K2, o[6], o[7], o[8]);
         tmem_wait(zb);
         // the accumulator has been read: the next product runs during the last piece's work
         tc_fence_before();
         __syncwarp();
-        if ((tid & 31) == 0) mbar_arrive(empty);
-        if (tid == 0 && it + 1 < my_tiles)
-            next_ok = mbar_wait_bounded(empty, (uint32_t)(it & 1), kMaxPolls) && issue_mma(it + 1);
-        bucket_piece(zb, Mb, K0, K1, K2, rec, 3, store);
+        if ((tid & 31) == 0 && it + 1 < my_tiles && (atom_add_acq_rel(readers, 1u) & 3u) == 3u)
+            issue_mma(it + 1);
+        bucket_piece(zb, Mb, K0, K1, K2, o[9], o[10], o[11]);
         if (v < n_vec) {
+            st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
+            st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
+            st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));
             norms[v] = nrm;
             scales[v] = scale;
         }
     }
-    if (fault && tid == 0) {
-        atomicOr(&g_fault, 8u);
-        // give what is still in flight a bounded chance to land before the memory goes away
-        for (int64_t i = n_landed; i < n_loaded; ++i) mbar_wait_bounded(full, (uint32_t)(i & 1), kMaxPolls);
-        if (n_mma > n_done) mbar_wait_bounded(done, (uint32_t)(n_done & 1), kMaxPolls);
-    }
+    if (fault && (tid & 31) == 0) atomicOr(&g_fault, 8u);
     tc_fence_before();
+    __syncthreads();
+    if (__syncthreads_or(fault) && tid == 0) {
+        // give what may still be in flight a bounded chance to land before the memory goes away
+        if (n_loaded > 0) mbar_wait_bounded(full, (uint32_t)((n_loaded - 1) & 1), kMaxPolls);
+        const uint32_t n_mma = *issued;
+        if (n_mma > 0) mbar_wait_bounded(done, (n_mma - 1) & 1u, kMaxPolls);
+    }
     __syncthreads();
     if (threadIdx.x < 32) {
         tc_fence_after();
