@@ -69,6 +69,23 @@ bool ensure_dynamic_smem(const void *kernel, size_t smem);
 int blocks_per_sm_cached(const void *kernel, int threads, size_t smem);
 inline int dtype_size(int t) { return t == WQ_F32 ? 4 : 2; }
 
+// Launch with programmatic stream serialization allowed (see pdl_wait / pdl_trigger).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*k)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, static_cast<KArgs>(args)...);
+}
+
 }  // namespace wq
 
 // ---------------------------------------------------------------------------------------------
@@ -184,6 +201,14 @@ __device__ __forceinline__ void tma_store_commit_wait_read() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+// Programmatic dependent launch. A kernel launched with launch_pdl may start while the kernel
+// before it on the stream is finishing; it must execute pdl_wait before it reads or writes global
+// memory that the earlier kernel could touch (pdl_wait returns once that kernel has completed and
+// its memory operations are visible; it returns at once when there is no such dependency).
+// pdl_trigger lets the next such kernel be scheduled as soon as every CTA of this one has issued it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Make generic-proxy shared-memory writes visible to the async (TMA) proxy.
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 

@@ -297,6 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // everything above touched only this CTA's resources and the constant table: from here on the
+    // kernel reads the input and writes the outputs, so the previous kernel must be complete
+    pdl_wait();
     const uint32_t tmem = *tslot + (uint32_t)(grp * kTile);  // this group's 128 columns
     const uint32_t my_lanes = tmem + ((uint32_t)(warp * 32) << 16);
 
@@ -345,6 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // the product has consumed the operand buffer: the next tile lands during this epilogue
         if (tid == 0 && it + 1 < my_tiles) issue_load(it + 1);
+        // on a group's last tile the block lets the next kernel in the stream be scheduled: its
+        // set-up overlaps this kernel's tail (it still waits for this kernel to finish before reading)
+        if (it + 1 == my_tiles) pdl_trigger();
         tc_fence_after();
 
         // pass 1: ||x||^2 = ||z||^2 / 128 (Parseval) and max|z|
@@ -458,7 +464,10 @@ wq_status launch(K k, int64_t cnt, const CUtensorMap &tm, const SignMask &m, uin
     const int64_t triples = (tiles + kGroups - 1) / kGroups;
     const int64_t g_ = sm_count() > 0 ? sm_count() : 1;
     const int64_t g = g_ < triples ? g_ : triples;
-    k<<<(unsigned)g, kThreads, kSmem, s>>>(cnt, tm, m, pc, nc, sc);
+    if (launch_pdl(k, (unsigned)g, kThreads, kSmem, s, cnt, tm, m, pc, nc, sc) != cudaSuccess) {
+        cudaGetLastError();
+        return WQ_ERR_CUDA;
+    }
     return launch_status();
 }
 }  // namespace

@@ -372,8 +372,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
     const float post = tq3::fwht_post();
 
     int64_t tile = blockIdx.x;
+    pdl_wait();  // the records may come from the kernel before this one
     Rec cur = load_rec(packed, norms, scales, n_vec, tile * kTile + tid);
     for (int it = 0; tile < n_tiles; ++it, tile += gridDim.x) {
+        // on its last tile the block lets the next kernel in the stream be scheduled: its set-up
+        // overlaps this kernel's tail (it still waits for this kernel to finish before reading)
+        if (tile + gridDim.x >= n_tiles) pdl_trigger();
         const Rec nxt = load_rec(packed, norms, scales, n_vec, (tile + gridDim.x) * kTile + tid);
         unsigned char *buf = obuf + (it % G::kBufs) * G::kTileBytes;
         if (tid == 0) bulk_wait_read<G::kBufs - 1>();  // the store that last read this buffer is done
