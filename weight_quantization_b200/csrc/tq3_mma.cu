@@ -353,16 +353,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it + 1 == my_tiles) pdl_trigger();
         tc_fence_after();
 
-        // pass 1: ||x||^2 = ||z||^2 / 128 (Parseval) and max|z|
+        // pass 1: ||x||^2 = ||z||^2 / 128 (Parseval) and max|z|. The pieces alternate between two
+        // register sets, so each piece's read from tensor memory overlaps the previous piece's work;
+        // the first piece of pass 2 is read while the per-vector scalars are formed.
         f32x2 acc[4] = {0ull, 0ull, 0ull, 0ull};
         float mm[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            float z[32];
-            tmem_ld32(my_lanes + 32 * c, z);
-            tmem_wait(z);
-            acc_piece(z, acc, mm);
-        }
+        float za[32], zb[32];
+        tmem_ld32(my_lanes + 0, za);
+        tmem_wait(za);
+        tmem_ld32(my_lanes + 32, zb);
+        acc_piece(za, acc, mm);
+        tmem_wait(zb);
+        tmem_ld32(my_lanes + 64, za);
+        acc_piece(zb, acc, mm);
+        tmem_wait(za);
+        tmem_ld32(my_lanes + 96, zb);
+        acc_piece(za, acc, mm);
+        tmem_wait(zb);
+        tmem_ld32(my_lanes + 0, za);
+        acc_piece(zb, acc, mm);
         float n2;
         {
             float a0, a1;
@@ -395,14 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float M = __uint_as_float(Mb);
         const float K0 = -__fmul_rn(t0, M), K1 = -__fmul_rn(t1, M), K2 = -__fmul_rn(t2, M);
 
-        // pass 2: the indices, 32 columns at a time
+        // pass 2: the indices, 32 columns at a time, the reads alternating as in pass 1
         const int64_t v = (stream + it * n_streams) * kTile + tid;
         uint8_t *const rec = packed + v * 48;
         uint32_t o[12];
-        // the pieces alternate between two register sets, so each piece's read from tensor
-        // memory overlaps the previous piece's work
-        float za[32], zb[32];
-        tmem_ld32(my_lanes + 0, za);
         tmem_wait(za);
         tmem_ld32(my_lanes + 32, zb);
         bucket_piece(za, Mb, K0, K1, K2, o[0], o[1], o[2]);
