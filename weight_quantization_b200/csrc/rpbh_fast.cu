@@ -188,6 +188,11 @@ __global__ void __launch_bounds__(kMaxThreads)
 // ---------------------------------------------------------------------------------------------
 struct Edges {
     float e[15];  // (c_k + c_{k+1}) / 2
+    // for an antisymmetric codebook, the positive edges e[L/2 .. L-2] as exact steps (see
+    // step_count): M[i] = 2^(24 - E) with E the binary exponent of the edge, K[i] = -edge * M[i];
+    // steps = 1 when every positive edge is at least 2^-103 (so that M is a normal fp32 value)
+    float M[7], K[7];
+    int steps;
 };
 
 __device__ __forceinline__ double block_sum_f64(double v, double *red) {
@@ -203,6 +208,46 @@ __device__ __forceinline__ double block_sum_f64(double v, double *red) {
     }
     __syncthreads();
     return red[32];
+}
+
+// a * b + c on both lanes, rounded up / down.
+__device__ __forceinline__ f32x2 fma_rp2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rp.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f32x2 fma_rm2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// The codes of two quotients u (both lanes) for an antisymmetric codebook with E.steps set, as
+// fp32 values 2^23 + code (the code is the value's low byte). The same decisions as bucketize<.., true>:
+// a' = |u| - u 2^-24 rounded up (|u| for u > 0, next(|u|) for u <= 0) is compared with the positive
+// edges strictly, each compare an exact 0/1 step sat(a' M + K) (a' > e means a' >= e + ulp, and
+// M = 2 / ulp(e)); with c the number of edges below a', the code is mid + 1/2 + sgn (c + 1/2),
+// sgn the sign of u + (-0) rounded down, which is -0 for both zeros (the page gives zero the
+// code below the middle edge).
+template <int BITS>
+__device__ __forceinline__ f32x2 sym_codes(f32x2 u, const Edges &E) {
+    constexpr int L = 1 << BITS, kPos = L / 2 - 1;
+    float u0, u1;
+    upk2(u, u0, u1);
+    const f32x2 ap = fma_rp2(u, pk2(-0x1p-24f, -0x1p-24f), pk2(fabsf(u0), fabsf(u1)));
+    float a0, a1;
+    upk2(ap, a0, a1);
+    f32x2 c = pk2(0.5f, 0.5f);
+#pragma unroll
+    for (int i = 0; i < kPos; ++i)
+        c = add2(c, pk2(__saturatef(__fmaf_rn(a0, E.M[i], E.K[i])), __saturatef(__fmaf_rn(a1, E.M[i], E.K[i]))));
+    float b0, b1, c0, c1;
+    upk2(fma_rm2(u, pk2(1.0f, 1.0f), pk2(-0.0f, -0.0f)), b0, b1);
+    upk2(c, c0, c1);
+    const f32x2 sc = pk2(__uint_as_float(__float_as_uint(c0) | (__float_as_uint(b0) & 0x80000000u)),
+                         __uint_as_float(__float_as_uint(c1) | (__float_as_uint(b1) & 0x80000000u)));
+    constexpr float kBase = 8388608.0f + (float)(L / 2 - 1);  // 2^23 + mid
+    return add2(add2(sc, pk2(0.5f, 0.5f)), pk2(kBase, kBase));
 }
 
 // bucketize(u, edges, right=False): the number of edges strictly below u.
@@ -680,6 +725,160 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     }
 }
 
+// Warp-local form of quantize_persistent, for h-blocks of at most 32 x 32 (S <= 32): warp w always
+// owns the same h-blocks, groups g = w, w + nwarps, ... of 32 / S blocks each, in every row. Both
+// butterfly passes of a block, its codes and their packing stay inside the owning warp (its part
+// of the transpose buffer is private), so a row needs one CTA barrier, for the norm; the partial
+// sums alternate between two sets by row, so a set is rewritten only after the barrier between.
+// A timed-out wait sets the fault flag but ends no thread's loop early, so every thread meets
+// every barrier.
+template <int B, bool kBf16, int BITS, bool kSym>
+__global__ void __launch_bounds__(kMaxThreads, 2)
+    quantize_warp(const void *__restrict__ w, int rows, int d, float post, const int32_t *__restrict__ perm,
+                  const int8_t *__restrict__ signs, Edges E, uint8_t *__restrict__ packed,
+                  void *__restrict__ row_norms) {
+    using G = Geo<B>;
+    constexpr int S = G::S, H = G::H;
+    constexpr int kBpw = 32 / S;    // blocks a warp works on at once: lane = sub-block * S + row / column
+    constexpr int kSlots = 64 / S;  // register slots per lane (the host checks the warp's share fits)
+    constexpr int esz = kBf16 ? 2 : 4;
+    static_assert(S <= 32, "a block's rows must fit one warp");
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ double red[2][kMaxThreads / 32];
+    unsigned char *base = align16(smem_raw);
+    const PLayout Lo(d, esz);
+    const uint16_t *perm16 = reinterpret_cast<const uint16_t *>(base + Lo.perm);
+    const uint32_t *sbits = reinterpret_cast<const uint32_t *>(base + Lo.bits);
+    unsigned char *const rb0 = base + Lo.row0;  // row buffers rb0 and rb0 + row_bytes
+    unsigned char *buf = base + Lo.buf;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + Lo.bar);
+    const uint32_t row_bytes = (uint32_t)d * esz;
+    const unsigned char *wb = static_cast<const unsigned char *>(w);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = (int)(blockDim.x >> 5);
+    const int sub = lane / S, rc = lane % S;
+    const int nb = d / H, ngroups = (nb + kBpw - 1) / kBpw;
+    int row = blockIdx.x;
+    if (!persistent_prologue(Lo, base, perm, signs, d, row < rows ? wb + (int64_t)row * row_bytes : nullptr,
+                             row_bytes))
+        return;
+    bool fault = false;
+    int last_buf = -1;  // thread 0: the buffer and phase of the last row copy it issued
+    uint32_t last_par = 0;
+    for (int it = 0; row < rows; ++it, row += gridDim.x) {
+        const int cur = it & 1;
+        const int nrow = row + gridDim.x;
+        // every thread passed the previous row's barrier after its last read of the other buffer
+        if (threadIdx.x == 0 && nrow < rows && !fault) {
+            mbar_expect_tx(&bar[cur ^ 1], row_bytes);
+            bulk_load((rb0 + (cur ^ 1) * row_bytes), wb + (int64_t)nrow * row_bytes, row_bytes, &bar[cur ^ 1]);
+            last_buf = cur ^ 1;
+            last_par = (uint32_t)(((it + 1) >> 1) & 1);
+        }
+        if (!fault && !mbar_wait_bounded(&bar[cur], (it >> 1) & 1, kMaxPolls)) {
+            fault = true;
+            atomicOr(&g_fault, 2u);
+        }
+        const unsigned char *rbc = rb0 + cur * row_bytes;
+        // pass 0 and pass 1 of the warp's blocks; w_rot stays in registers
+        float zk[kSlots][S];
+        double ss = 0.0;
+#pragma unroll
+        for (int k = 0; k < kSlots; ++k) {
+            const int g = warp + k * nwarps;
+            const int blk = g * kBpw + sub;
+            if (g < ngroups) {  // warp-uniform
+                if (blk < nb) {
+                    float y[S];
+                    gather_row_smem<B, kBf16>(y, rbc, blk * H + rc * S, perm16, sbits);
+                    store_row<B>(buf, y, blk, rc);
+                }
+                __syncwarp();
+                if (blk < nb) {
+                    load_col<B>(zk[k], buf, blk, rc);
+                    butterfly<S>(zk[k]);
+#pragma unroll
+                    for (int t = 0; t < S; ++t) {
+                        zk[k][t] = __fmul_rn(zk[k][t], post);
+                        const double dz = (double)zk[k][t];
+                        ss = __fma_rn(dz, dz, ss);
+                    }
+                }
+            }
+        }
+        // rho = ||w_rot||: every lane of a warp gets the same warp sum, every thread the same total
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss = __dadd_rn(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+        if (lane == 0) red[cur][warp] = ss;
+        fence_proxy_async_smem();  // this thread's reads of the row buffer precede the copy that refills it
+        __syncthreads();
+        double tot = 0.0;
+        for (int v = 0; v < nwarps; ++v) tot = __dadd_rn(tot, red[cur][v]);
+        const float rho = __double2float_rn(__dsqrt_rn(tot));
+        const float den = __fadd_rn(rho, 1e-10f);
+        const float rden = __frcp_rn(den);
+        // codes, one byte each in element order, into the block's own part of the transpose buffer
+        // (its columns are in registers by now); u = z / den correctly rounded (Markstein:
+        // q0 = RN(z r), r = RN(1 / den), the remainder z - q0 den exact, u = RN(q0 + rem r)), two
+        // elements at a time
+        const f32x2 RDEN = pk2(rden, rden), NDEN = pk2(-den, -den);
+#pragma unroll
+        for (int k = 0; k < kSlots; ++k) {
+            const int g = warp + k * nwarps;
+            const int blk = g * kBpw + sub;
+            if (g < ngroups && blk < nb) {
+                unsigned char *cb = buf + 4 * blk * H + rc;
+#pragma unroll
+                for (int t = 0; t < S; t += 2) {
+                    const f32x2 z = pk2(zk[k][t], zk[k][t + 1]);
+                    const f32x2 q0 = mul2(z, RDEN);
+                    const f32x2 u = fma2(fma2(q0, NDEN, z), RDEN, q0);
+                    if constexpr (kSym) {
+                        float v0, v1;
+                        upk2(sym_codes<BITS>(u, E), v0, v1);
+                        cb[t * S] = (uint8_t)__float_as_uint(v0);
+                        cb[(t + 1) * S] = (uint8_t)__float_as_uint(v1);
+                    } else {
+                        float u0, u1;
+                        upk2(u, u0, u1);
+                        cb[t * S] = (uint8_t)bucketize<BITS, false>(u0, E);
+                        cb[(t + 1) * S] = (uint8_t)bucketize<BITS, false>(u1, E);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        // pack_codes: the warp's groups of 32 codes (S of them per block group), one per lane
+        uint8_t *dst = packed + ((int64_t)row * d / 8) * BITS;
+#pragma unroll
+        for (int k = 0; k < kSlots; ++k) {
+            const int g = warp + k * nwarps;
+            if (g < ngroups && lane < S) {
+                const int blk = g * kBpw + lane / (H / 32), q = lane % (H / 32);
+                if (blk < nb) {
+                    const unsigned char *src = buf + 4 * blk * H + 32 * q;
+                    const uint4 c0 = *reinterpret_cast<const uint4 *>(src);
+                    const uint4 c1 = *reinterpret_cast<const uint4 *>(src + 16);
+                    const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                    uint32_t word[BITS];
+                    pack32<BITS>(cw, word);
+                    uint32_t *out = reinterpret_cast<uint32_t *>(dst + (blk * H + 32 * q) / 8 * BITS);
+#pragma unroll
+                    for (int j = 0; j < BITS; ++j) out[j] = __byte_perm(word[j], 0, 0x0123);
+                }
+            }
+        }
+        __syncwarp();  // the codes are read before the next row's pass 0 rewrites this part of the buffer
+        if (threadIdx.x == 0) {
+            if (kBf16)
+                static_cast<uint16_t *>(row_norms)[row] = f32_to_bf16(rho);
+            else
+                static_cast<float *>(row_norms)[row] = rho;
+        }
+    }
+    // a fault may leave thread 0's last row copy in flight: give it a bounded chance to land
+    if (fault && threadIdx.x == 0 && last_buf >= 0) mbar_wait_bounded(&bar[last_buf], last_par, kMaxPolls);
+}
+
 // ---------------------------------------------------------------------------------------------
 // host dispatch
 // ---------------------------------------------------------------------------------------------
@@ -805,6 +1004,24 @@ wq_status quantize_b(const void *w, int64_t rows, int64_t d, const int32_t *perm
     auto k = quantize_kernel<B, kBf16, BITS, kSym>;
     wq_status st = prep(k, smem);
     if (st != WQ_OK) return st;
+    // the warp-local form (where its register-resident slots compile without spilling): each warp's
+    // share of block groups must fit its 64 / S register slots
+    if constexpr (B == 5 || (B == 4 && kBf16)) {
+        constexpr int64_t S = int64_t(1) << B;
+        const int64_t groups = ((d >> (2 * B)) + 32 / S - 1) / (32 / S);
+        if ((!kSym || E.steps) && persistent_fits(d, kBf16 ? 2 : 4) &&
+            (groups + threads / 32 - 1) / (threads / 32) <= 64 / S) {
+            const size_t psmem = pers_smem(d, kBf16 ? 2 : 4);
+            auto kw = quantize_warp<B, kBf16, BITS, kSym>;
+            st = prep(kw, psmem);
+            if (st != WQ_OK) return st;
+            if (blocks_per_sm(reinterpret_cast<const void *>(kw), threads, psmem) >= 1) {
+                kw<<<persistent_grid(kw, threads, psmem, rows), threads, psmem, s>>>(
+                    w, (int)rows, (int)d, fwht_post(d & -d), perm, signs, E, packed, row_norms);
+                return launch_status();
+            }
+        }
+    }
     // the persistent form keeps each thread's slots of the row in registers: at most 64 / S of them
     if (persistent_fits(d, kBf16 ? 2 : 4) && (d >> B) <= (int64_t)(64 >> B) * threads) {
         const size_t psmem = pers_smem(d, kBf16 ? 2 : 4);
@@ -855,6 +1072,20 @@ wq_status quantize(const void *w, int w_dtype, int64_t rows, int64_t d, const in
     for (int k = 0; k < L; ++k)
         if (!(codebook[k] == -codebook[L - 1 - k])) sym = false;
     if (sym && !(E.e[L / 2 - 1] == 0.0f)) sym = false;
+    if (sym) {
+        E.steps = 1;
+        for (int i = 0; i < L / 2 - 1; ++i) {
+            const float e = E.e[L / 2 + i];
+            int ex = 0;
+            std::frexp(e, &ex);  // e = f 2^ex, f in [0.5, 1): binary exponent ex - 1
+            if (!(e >= 0x1p-103f) || !std::isfinite(e)) {
+                E.steps = 0;
+                break;
+            }
+            E.M[i] = std::ldexp(1.0f, 25 - ex);
+            E.K[i] = -e * E.M[i];  // exact: e scaled by a power of two into [2^24, 2^25)
+        }
+    }
     const bool bf = w_dtype == WQ_BF16;
     switch (log2_block(d) / 2) {
         case 3: return quantize_sym<3>(bf, sym, bits, w, rows, d, perm, signs, E, packed, row_norms, s);
