@@ -292,6 +292,22 @@ __device__ __forceinline__ void pack32(const uint32_t (&cw)[8], uint32_t (&word)
         }
     }
 }
+// pack32 for BITS = 3 with the codes combined four at a time: byte-reversed word r = c0 c1 c2 c3;
+// (r | r >> 5) & 0x003F003F holds c0 c1 at bits 16 .. 21 and c2 c3 at bits 0 .. 5, and one more
+// shift and mask gives the 12-bit chunk c0 c1 c2 c3 (MSB first); eight chunks make the three words.
+__device__ __forceinline__ void pack32_b3(const uint32_t (&cw)[8], uint32_t (&word)[3]) {
+    uint32_t ch[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t r = __byte_perm(cw[j], 0u, 0x0123);
+        const uint32_t t = (r | (r >> 5)) & 0x003F003Fu;
+        ch[j] = (t >> 10) | (t & 0x3Fu);
+    }
+    word[0] = (ch[0] << 20) | (ch[1] << 8) | (ch[2] >> 4);
+    word[1] = (ch[2] << 28) | (ch[3] << 16) | (ch[4] << 4) | (ch[5] >> 8);
+    word[2] = (ch[5] << 24) | (ch[6] << 12) | ch[7];
+}
+
 // unpack_codes for one group: the inverse of pack32, code i into byte i of cw.
 template <int BITS>
 __device__ __forceinline__ void unpack32(const uint32_t (&word)[BITS], uint32_t (&cw)[8]) {
@@ -847,24 +863,27 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
             }
         }
         __syncwarp();
-        // pack_codes: the warp's groups of 32 codes (S of them per block group), one per lane
+        // pack_codes: the warp's groups of 32 codes (S per block group, over all its block groups)
+        // spread over the 32 lanes
         uint8_t *dst = packed + ((int64_t)row * d / 8) * BITS;
 #pragma unroll
-        for (int k = 0; k < kSlots; ++k) {
+        for (int j0 = 0; j0 < kSlots * S; j0 += 32) {
+            const int unit = j0 + lane, k = unit / S;
             const int g = warp + k * nwarps;
-            if (g < ngroups && lane < S) {
-                const int blk = g * kBpw + lane / (H / 32), q = lane % (H / 32);
-                if (blk < nb) {
-                    const unsigned char *src = buf + 4 * blk * H + 32 * q;
-                    const uint4 c0 = *reinterpret_cast<const uint4 *>(src);
-                    const uint4 c1 = *reinterpret_cast<const uint4 *>(src + 16);
-                    const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                    uint32_t word[BITS];
+            const int blk = g * kBpw + (unit % S) / (H / 32), q = (unit % S) % (H / 32);
+            if (k < kSlots && g < ngroups && blk < nb) {
+                const unsigned char *src = buf + 4 * blk * H + 32 * q;
+                const uint4 c0 = *reinterpret_cast<const uint4 *>(src);
+                const uint4 c1 = *reinterpret_cast<const uint4 *>(src + 16);
+                const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                uint32_t word[BITS];
+                if constexpr (BITS == 3)
+                    pack32_b3(cw, word);
+                else
                     pack32<BITS>(cw, word);
-                    uint32_t *out = reinterpret_cast<uint32_t *>(dst + (blk * H + 32 * q) / 8 * BITS);
+                uint32_t *out = reinterpret_cast<uint32_t *>(dst + (blk * H + 32 * q) / 8 * BITS);
 #pragma unroll
-                    for (int j = 0; j < BITS; ++j) out[j] = __byte_perm(word[j], 0, 0x0123);
-                }
+                for (int j = 0; j < BITS; ++j) out[j] = __byte_perm(word[j], 0, 0x0123);
             }
         }
         __syncwarp();  // the codes are read before the next row's pass 0 rewrites this part of the buffer
