@@ -51,7 +51,7 @@ def _quantize_and_check(wq, oracle, w, is_bf16, d, bits):
 
 
 @pytest.mark.parametrize("d,rows", [(32, 5), (96, 37), (192, 11), (256, 3), (1024, 9), (3072, 17), (640, 1),
-                                    (4096, 3), (12288, 2)])
+                                    (4096, 3), (12288, 2), (6400, 7)])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 @pytest.mark.parametrize("is_bf16", [False, True])
 def test_quantize_small(wq, oracle, d, rows, bits, is_bf16):
@@ -139,7 +139,7 @@ def test_quantize_then_dequantize_llm_roundtrip(wq, oracle):
 
 
 @pytest.mark.parametrize("rows,d", [(2048, 11008), (4096, 3072), (3, 96), (1, 32), (5, 192), (3, 4096),
-                                    (7, 640)])
+                                    (7, 640), (9, 2880), (5, 6400)])
 def test_rotate_activations(wq, oracle, rows, d):
     perm, signs, perm_d, signs_d = _params(d)
     h = d & -d
@@ -150,6 +150,15 @@ def test_rotate_activations(wq, oracle, rows, d):
     r = parity.rel_rows(oracle.bf16_array_to_f32(got), oracle.bf16_array_to_f32(ref))
     assert r.max() <= parity.BF16_RTOL
     assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("rows,d", [(6, 6400), (4, 2880)])
+def test_rotate_fp32_many_blocks(wq, oracle, rows, d):
+    """fp32 rotation of rows with many h-blocks (25 blocks of 256; 45 blocks of 64), bit for bit."""
+    perm, signs, perm_d, signs_d = _params(d)
+    x = torch.from_numpy(inputs.gaussian((rows, d), seed=d + rows)).cuda()
+    xr = wq.rpbh_rotate_activations(x, perm_d, signs_d)
+    assert np.array_equal(xr.cpu().numpy(), oracle.rpbh_forward(x.cpu().numpy(), perm, signs, d & -d))
 
 
 def test_rotate_fp32_and_matmul_invariance(wq, oracle):

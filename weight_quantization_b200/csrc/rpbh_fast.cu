@@ -898,6 +898,134 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
     if (fault && threadIdx.x == 0 && last_buf >= 0) mbar_wait_bounded(&bar[last_buf], last_par, kMaxPolls);
 }
 
+// Warp-local form of the activation rotation (S <= 32): warp w always owns the same h-blocks,
+// groups g = w, w + nwarps, ... of 32 / S blocks, and runs both butterfly passes of a group
+// through its own 128 S-byte transpose scratch; the outputs go from registers straight to global
+// memory (for each t, the S lanes of a block store S consecutive elements). Rows are
+// double-buffered by 1-D bulk copies; one CTA barrier per row tells thread 0 that every warp
+// has finished gathering from a row buffer, which then takes the row after next.
+struct RLayout {
+    int perm, bits, row0, row1, scr, bar, total;
+    __host__ __device__ RLayout(int d, int esz, int nwarps, int S) {
+        perm = 0;
+        bits = a16(2 * d);
+        row0 = bits + a16(d / 8);
+        row1 = row0 + d * esz;
+        scr = row1 + d * esz;
+        bar = scr + nwarps * 128 * S;
+        total = bar + 32;
+    }
+};
+
+constexpr int kRotWarps = 12;  // warps per CTA of rotate_warp (two CTAs per SM fit the register file)
+
+template <int B, bool kBf16>
+__global__ void __launch_bounds__(32 * kRotWarps, 2)
+    rotate_warp(const void *__restrict__ x, int rows, int d, float post, const int32_t *__restrict__ perm,
+                const int8_t *__restrict__ signs, void *__restrict__ out) {
+    using G = Geo<B>;
+    constexpr int S = G::S, H = G::H, kBpw = 32 / S;
+    constexpr int esz = kBf16 ? 2 : 4;
+    static_assert(S <= 32, "a block's rows must fit one warp");
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *base = align16(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = (int)(blockDim.x >> 5);
+    const RLayout Lo(d, esz, nwarps, S);
+    uint16_t *perm16 = reinterpret_cast<uint16_t *>(base + Lo.perm);
+    uint32_t *sbits = reinterpret_cast<uint32_t *>(base + Lo.bits);
+    unsigned char *const rb0 = base + Lo.row0;  // row buffers rb0 and rb0 + row_bytes
+    unsigned char *const scr = base + Lo.scr + warp * 128 * S;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + Lo.bar);
+    const uint32_t row_bytes = (uint32_t)d * esz;
+    const unsigned char *xb = static_cast<const unsigned char *>(x);
+    const int sub = lane / S, rc = lane % S;
+    const int nb = d / H, ngroups = (nb + kBpw - 1) / kBpw;
+
+    // tables: perm (int32) lands in the row buffers, the signs in the scratch; both are converted
+    // in place before the first row is fetched
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        mbar_init(&bar[2], 1);
+        mbar_expect_tx(&bar[2], 5u * (uint32_t)d);
+        bulk_load(rb0, perm, 4u * (uint32_t)d, &bar[2]);
+        bulk_load(base + Lo.scr, signs, (uint32_t)d, &bar[2]);
+    }
+    __syncthreads();
+    if (!row_ready(&bar[2], 0)) return;
+    {
+        const int32_t *p32 = reinterpret_cast<const int32_t *>(rb0);
+        for (int j = threadIdx.x; j < d; j += blockDim.x) perm16[j] = (uint16_t)clampi(p32[j], d);
+        const unsigned char *sg = base + Lo.scr;
+        for (int w = threadIdx.x; w < d / 32; w += blockDim.x) {
+            uint32_t bits = 0;
+            for (int t = 0; t < 32; ++t) bits |= (uint32_t)(((uint8_t)sg[32 * w + t]) >> 7) << t;
+            sbits[w] = bits;
+        }
+    }
+    fence_proxy_async_smem();  // these reads of the row buffers precede the copies that refill them
+    __syncthreads();
+    int row = blockIdx.x;
+    uint32_t n_iss0 = 0u, n_iss1 = 0u;  // thread 0: row copies issued into each buffer
+    if (threadIdx.x == 0)
+        for (int b = 0; b < 2; ++b) {
+            const int r = row + b * (int)gridDim.x;
+            if (r < rows) {
+                mbar_expect_tx(&bar[b], row_bytes);
+                bulk_load(rb0 + b * row_bytes, xb + (int64_t)r * row_bytes, row_bytes, &bar[b]);
+                if (b == 0) ++n_iss0; else ++n_iss1;
+            }
+        }
+    bool fault = false;
+    for (int it = 0; row < rows; ++it, row += gridDim.x) {
+        const int cur = it & 1;
+        if (!fault && !mbar_wait_bounded(&bar[cur], (it >> 1) & 1, kMaxPolls)) {
+            fault = true;
+            atomicOr(&g_fault, 2u);
+        }
+        const unsigned char *rbc = rb0 + cur * row_bytes;
+        unsigned char *orow = static_cast<unsigned char *>(out) + (int64_t)row * row_bytes;
+        for (int g = warp; g < ngroups; g += nwarps) {
+            const int blk = g * kBpw + sub;
+            if (blk < nb) {
+                float y[S];
+                gather_row_smem<B, kBf16>(y, rbc, blk * H + rc * S, perm16, sbits);
+                store_row<B>(scr, y, sub, rc);
+            }
+            __syncwarp();
+            if (blk < nb) {
+                float y[S];
+                load_col<B>(y, scr, sub, rc);
+                butterfly<S>(y);
+#pragma unroll
+                for (int t = 0; t < S; ++t) {
+                    const int j = blk * H + rc + t * S;
+                    const float z = __fmul_rn(y[t], post);
+                    if (kBf16)
+                        reinterpret_cast<uint16_t *>(orow)[j] = f32_to_bf16(z);
+                    else
+                        reinterpret_cast<float *>(orow)[j] = z;
+                }
+            }
+            __syncwarp();  // the columns are read before the warp's next group rewrites the scratch
+        }
+        // every warp has gathered from this buffer: it takes the row after next
+        fence_proxy_async_smem();
+        __syncthreads();
+        const int r2 = row + 2 * (int)gridDim.x;
+        if (threadIdx.x == 0 && r2 < rows && !fault) {
+            mbar_expect_tx(&bar[cur], row_bytes);
+            bulk_load(rb0 + cur * row_bytes, xb + (int64_t)r2 * row_bytes, row_bytes, &bar[cur]);
+            if (cur == 0) ++n_iss0; else ++n_iss1;
+        }
+    }
+    // a fault may leave row copies in flight: give the last one into each buffer a bounded chance
+    if (fault && threadIdx.x == 0) {
+        if (n_iss0 > 0) mbar_wait_bounded(&bar[0], (n_iss0 - 1) & 1u, kMaxPolls);
+        if (n_iss1 > 0) mbar_wait_bounded(&bar[1], (n_iss1 - 1) & 1u, kMaxPolls);
+    }
+}
+
 // ---------------------------------------------------------------------------------------------
 // host dispatch
 // ---------------------------------------------------------------------------------------------
@@ -988,6 +1116,24 @@ wq_status rotate_b(const void *x, int64_t rows, int64_t d, const int32_t *perm, 
     auto k = rotate_kernel<B, kBf16>;
     wq_status st = prep(k, smem);
     if (st != WQ_OK) return st;
+    // the warp-local form: kRotWarps warps, each with a 128 S-byte transpose scratch (which also
+    // stages the signs at set-up, so it must hold d bytes)
+    if constexpr (B <= 5) {
+        constexpr int S = 1 << B, kW = kRotWarps;
+        const size_t wsmem = (size_t)RLayout((int)d, kBf16 ? 2 : 4, kW, S).total + 16;
+        // (only when every warp has a block group of each row: with fewer, most warps would idle)
+        const int64_t groups = ((d >> (2 * B)) + 32 / S - 1) / (32 / S);
+        if (groups >= kW && d <= 32768 && (int64_t)kW * 128 * S >= d && wsmem + 1024 <= smem_limit()) {
+            auto kw = rotate_warp<B, kBf16>;
+            st = prep(kw, wsmem);
+            if (st != WQ_OK) return st;
+            if (blocks_per_sm(reinterpret_cast<const void *>(kw), 32 * kW, wsmem) >= 1) {
+                kw<<<persistent_grid(kw, 32 * kW, wsmem, rows), 32 * kW, wsmem, s>>>(
+                    x, (int)rows, (int)d, fwht_post(d & -d), perm, signs, out);
+                return launch_status();
+            }
+        }
+    }
     if (persistent_fits(d, kBf16 ? 2 : 4)) {
         const size_t psmem = pers_smem(d, kBf16 ? 2 : 4);
         auto kp = rotate_persistent<B, kBf16>;
