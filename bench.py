@@ -127,6 +127,31 @@ def traffic_bytes(kernel: str):
     return None
 
 
+def pipelined_step(n, chunks, streams, h2d, compute, d2h):
+    """One end-to-end step over n units in `chunks` pieces on three streams (copy in, kernels, copy
+    out): piece i is copied in, processed and copied out in that order, while the copy in of piece
+    i + 1 and the copy out of piece i - 1 overlap piece i's kernels (host-device copies run both
+    directions at once). The step starts after, and the caller's stream then waits for, all of it."""
+    s_in, s_c, s_out = streams
+    cur = torch.cuda.current_stream()
+    for s in streams:
+        s.wait_stream(cur)
+    for i in range(chunks):
+        a, b = i * n // chunks, (i + 1) * n // chunks
+        with torch.cuda.stream(s_in):
+            h2d(a, b)
+        s_c.wait_stream(s_in)
+        with torch.cuda.stream(s_c):
+            compute(a, b)
+        s_out.wait_stream(s_c)
+        with torch.cuda.stream(s_out):
+            d2h(a, b)
+    for s in streams:
+        cur.wait_stream(s)
+
+
+E2E_CHUNKS = 8
+
 # ---------------------------------------------------------------------------------------------
 # workloads
 # ---------------------------------------------------------------------------------------------
@@ -184,13 +209,34 @@ class KVWorkload:
         self.h2d = sum(t.numel() * t.element_size() for t in self.pin_in)
         self.d2h = sum(t.numel() * t.element_size() for t in self.pin_out + self.pin_packed + self.pin_ns)
 
+        self.streams = [torch.cuda.Stream(self.x[0].device) for _ in range(3)]
+
     def e2e_step(self):
-        self.x[0].copy_(self.pin_in[0], non_blocking=True)
-        self.step()
-        self.pin_out[0].copy_(self.out[0], non_blocking=True)
-        self.pin_packed[0].copy_(self.packed[0], non_blocking=True)
-        self.pin_ns[0][0].copy_(self.norms[0], non_blocking=True)
-        self.pin_ns[0][1].copy_(self.scales[0], non_blocking=True)
+        """The cache in from pinned memory, encoded and decoded through the public calls, the
+        decoded cache and the records out, in E2E_CHUNKS pieces pipelined over three streams."""
+        o = self.ops
+
+        def h2d(a, b):
+            self.x[0][a:b].copy_(self.pin_in[0][a:b], non_blocking=True)
+
+        def compute(a, b):
+            o.tq3_encode(self.x[0][a:b], self.mask, self.packed[0][a:b].view(-1, 1, 48),
+                         self.norms[0][a:b].view(-1, 1), self.scales[0][a:b].view(-1, 1))
+            o.tq3_decode(self.packed[0][a:b], self.norms[0][a:b], self.scales[0][a:b], self.mask,
+                         out=self.out[0][a:b])
+
+        def d2h(a, b):
+            self.pin_out[0][a:b].copy_(self.out[0][a:b], non_blocking=True)
+            self.pin_packed[0][a:b].copy_(self.packed[0][a:b], non_blocking=True)
+            self.pin_ns[0][0][a:b].copy_(self.norms[0][a:b], non_blocking=True)
+            self.pin_ns[0][1][a:b].copy_(self.scales[0][a:b], non_blocking=True)
+
+        pipelined_step(self.units, E2E_CHUNKS, self.streams, h2d, compute, d2h)
+
+    def e2e_check(self):
+        """After the timed region: the host copies equal the device results."""
+        return (torch.equal(self.pin_out[0], self.out[0].cpu()) and torch.equal(self.pin_packed[0], self.packed[0].cpu())
+                and torch.equal(self.pin_ns[0][0], self.norms[0].cpu()) and torch.equal(self.pin_ns[0][1], self.scales[0].cpu()))
 
     # the oracle on a bounded sample of the same cache
     def oracle_rate(self, budget_s=10.0):
@@ -240,14 +286,27 @@ class LongContextWorkload(KVWorkload):
         self.pin_out = torch.empty(self.n_half, 128, dtype=torch.bfloat16).pin_memory()
         self.h2d = sum(t.numel() * t.element_size() for t in self.pin_rec)
         self.d2h = self.pin_out.numel() * 2
+        self.streams = [torch.cuda.Stream(self.out.device) for _ in range(3)]
 
     step = KVWorkload.step
 
     def e2e_step(self):
-        for d, h in zip(self.rec, self.pin_rec):
-            d.copy_(h, non_blocking=True)
-        self.step()
-        self.pin_out.copy_(self.out, non_blocking=True)
+        """The records in from pinned memory, decoded through the public call, the bf16 cache out,
+        in E2E_CHUNKS pieces pipelined over three streams."""
+        def h2d(a, b):
+            for d, h in zip(self.rec, self.pin_rec):
+                d[a:b].copy_(h[a:b], non_blocking=True)
+
+        def compute(a, b):
+            self.ops.tq3_decode(self.rec[0][a:b], self.rec[1][a:b], self.rec[2][a:b], self.mask, out=self.out[a:b])
+
+        def d2h(a, b):
+            self.pin_out[a:b].copy_(self.out[a:b], non_blocking=True)
+
+        pipelined_step(self.units, E2E_CHUNKS, self.streams, h2d, compute, d2h)
+
+    def e2e_check(self):
+        return torch.equal(self.pin_out, self.out.cpu())
 
     def oracle_rate(self, budget_s=10.0):
         import oracle
@@ -481,6 +540,8 @@ def run_ours(args):
     ee.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(es.elapsed_time(ee), world)
+    if hasattr(wl, "e2e_check") and not wl.e2e_check():
+        raise RuntimeError("end-to-end step: the host copies differ from the device results")
     e2e_value = world * wl.units * e2e_steps / (e2e_ms / 1e3)
 
     cpu = None
