@@ -51,7 +51,7 @@ def _quantize_and_check(wq, oracle, w, is_bf16, d, bits):
 
 
 @pytest.mark.parametrize("d,rows", [(32, 5), (96, 37), (192, 11), (256, 3), (1024, 9), (3072, 17), (640, 1),
-                                    (4096, 3), (12288, 2), (6400, 7)])
+                                    (4096, 3), (12288, 2), (6400, 7), (9472, 5)])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 @pytest.mark.parametrize("is_bf16", [False, True])
 def test_quantize_small(wq, oracle, d, rows, bits, is_bf16):
