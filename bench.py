@@ -174,31 +174,45 @@ class KVWorkload:
         n = self.units
         self.mask = ops.sign_mask_words(inputs.tq3_sign_bits())
         self.x = [self.host[0].to(dev)]
-        self.packed = [torch.empty(n, 48, dtype=torch.uint8, device=dev)]
-        self.norms = [torch.empty(n, dtype=torch.float32, device=dev)]
-        self.scales = [torch.empty(n, dtype=torch.float32, device=dev)]
+        # The records (29 MB, smaller than L2) rotate over RSETS sets: launch or step k encodes into
+        # set k and decodes set k + 1, written RSETS - 1 launches earlier, so no decode reads
+        # records that are still in L2 (the 134 MB cache itself is larger than L2).
+        R = self.RSETS
+        self.packed = [torch.empty(n, 48, dtype=torch.uint8, device=dev) for _ in range(R)]
+        self.norms = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(R)]
+        self.scales = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(R)]
         self.out = [torch.empty(n, 128, dtype=torch.bfloat16, device=dev)]
+        for k in range(R):
+            self._encode(k)
         self.kernels = ["tq3_encode", "tq3_decode"]
         self.bytes_per_launch = {"tq3_encode": 312 * n, "tq3_decode": 312 * n}
+        self.l2 = (f"cache (134 MB) larger than L2; records rotate over {R} sets: launch k encodes into "
+                   f"set k % {R} and decodes set (k + 1) % {R}, written {R - 1} launches earlier")
 
-    def _encode(self, exact=False):
-        self.ops.tq3_encode(self.x[0], self.mask, self.packed[0].view(-1, 1, 48), self.norms[0].view(-1, 1),
-                            self.scales[0].view(-1, 1), exact=exact)
+    RSETS = 8
+    rotation = RSETS  # the buffer choice repeats every `rotation` steps
 
-    def _decode(self):
-        self.ops.tq3_decode(self.packed[0], self.norms[0], self.scales[0], self.mask, out=self.out[0])
+    def _encode(self, k, exact=False):
+        r = k % self.RSETS
+        self.ops.tq3_encode(self.x[0], self.mask, self.packed[r].view(-1, 1, 48), self.norms[r].view(-1, 1),
+                            self.scales[r].view(-1, 1), exact=exact)
+
+    def _decode(self, k):
+        r = (k + 1) % self.RSETS
+        self.ops.tq3_decode(self.packed[r], self.norms[r], self.scales[r], self.mask, out=self.out[0])
 
     def parts(self):
-        """(kernel, launches, fn) in step order: encode the cache, then decode it."""
+        """(kernel, launches, fn(k)) in step order: encode the cache, then decode it; k is the step
+        (or launch) index, which picks the rotating buffers."""
         return [("tq3_encode", 1, self._encode), ("tq3_decode", 1, self._decode)]
 
     def extras(self):
         """Kernels timed beside the step (not part of it): the bit-exact encoder on the same cache."""
-        return [("tq3_encode_exact", 1, lambda: self._encode(exact=True))]
+        return [("tq3_encode_exact", 1, lambda k: self._encode(k, exact=True))]
 
-    def step(self):
+    def step(self, k=0):
         for _, _, fn in self.parts():
-            fn()
+            fn(k)
 
     # end to end: pinned host cache in; decoded cache and the TQ3 records out
     def e2e_setup(self):
@@ -267,16 +281,25 @@ class LongContextWorkload(KVWorkload):
         p, n, s = inputs.long_context_records(seed=seed)
         self.mask = ops.sign_mask_words(inputs.tq3_sign_bits())
         self.host_rec = (torch.from_numpy(p), torch.from_numpy(n), torch.from_numpy(s))
-        self.rec = [t.to(dev) for t in self.host_rec]
+        # the records (59 MB, smaller than L2) rotate over RSETS copies, one per launch
+        self.recs = [[t.to(dev) for t in self.host_rec] for _ in range(self.RSETS)]
+        self.rec = self.recs[0]
         self.n_half = p.shape[0]
         self.units = self.n_half
         self.out = torch.empty(self.n_half, 128, dtype=torch.bfloat16, device=dev)
         self.kernels = ["tq3_decode"]
         self.bytes_per_launch = {"tq3_decode": 312 * self.n_half}
+        self.l2 = (f"records rotate over {self.RSETS} copies ({self.RSETS} x 59 MB, larger than L2), launch k "
+                   f"decoding copy k % {self.RSETS}")
+
+    RSETS = 4
+    rotation = RSETS
 
     def parts(self):
-        return [("tq3_decode", 1, lambda: self.ops.tq3_decode(self.rec[0], self.rec[1], self.rec[2], self.mask,
-                                                               out=self.out))]
+        def dec(k):
+            r = self.recs[k % self.RSETS]
+            self.ops.tq3_decode(r[0], r[1], r[2], self.mask, out=self.out)
+        return [("tq3_decode", 1, dec)]
 
     def extras(self):
         return []
@@ -338,31 +361,53 @@ class RPBHWorkload:
         self.rows, self.d, self.xrows, self.bits = rows, d, xrows, bits
         bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
         self.host = [bf(w), bf(x)]
-        self.w, self.x = (t.to(dev) for t in self.host)
+        # W (75-90 MB), x (25-45 MB) and the codes (14-17 MB) are smaller than L2: each rotates over
+        # copies, so a launch reads data last touched several hundred MB of traffic earlier
+        W, X, P = self.WSETS, self.XSETS, self.PSETS
+        self.ws = [self.host[0].to(dev) for _ in range(W)]
+        self.xs = [self.host[1].to(dev) for _ in range(X)]
+        self.w, self.x = self.ws[0], self.xs[0]
         self.perm = torch.from_numpy(perm).to(dev)
         self.signs = torch.from_numpy(signs).to(dev)
         self.cb = ops.rpbh_codebook(bits, d)
-        self.packed = torch.empty(ops.rpbh_packed_bytes(rows, d, bits), dtype=torch.uint8, device=dev)
-        self.norms = torch.empty(rows, dtype=torch.bfloat16, device=dev)
+        self.packeds = [torch.empty(ops.rpbh_packed_bytes(rows, d, bits), dtype=torch.uint8, device=dev)
+                        for _ in range(P)]
+        self.normss = [torch.empty(rows, dtype=torch.bfloat16, device=dev) for _ in range(P)]
+        self.packed, self.norms = self.packeds[0], self.normss[0]
         self.wq = torch.empty(rows, d, dtype=torch.bfloat16, device=dev)
         self.xr = torch.empty(xrows, d, dtype=torch.bfloat16, device=dev)
+        for k in range(P):
+            self._quantize(k)
         self.units = rows * d
         self.kernels = ["rpbh_quantize", "rpbh_dequantize", "rpbh_rotate"]
         n = rows * d
         self.bytes_per_launch = {"rpbh_quantize": 2 * n + n * bits // 8 + 2 * rows,
                                  "rpbh_dequantize": 2 * n + n * bits // 8 + 2 * rows,
                                  "rpbh_rotate": 4 * xrows * d}
+        self.l2 = (f"W rotates over {W} copies, x over {X}, the codes over {P} sets: launch k quantizes W "
+                   f"copy k % {W} into set k % {P}, dequantizes set (k + 1) % {P} (written {P - 1} launches "
+                   f"earlier) and rotates x copy k % {X}")
+
+    WSETS, XSETS, PSETS = 3, 4, 3
+    rotation = 12  # lcm of the three
+
+    def _quantize(self, k):
+        p = k % self.PSETS
+        self.ops.rpbh_quantize_weight(self.ws[k % self.WSETS], self.perm, self.signs, self.bits, self.cb,
+                                      self.packeds[p], self.normss[p])
 
     def parts(self):
         o = self.ops
-        return [
-            ("rpbh_quantize", 1, lambda: o.rpbh_quantize_weight(self.w, self.perm, self.signs, self.bits, self.cb,
-                                                                self.packed, self.norms)),
-            ("rpbh_rotate", 1, lambda: o.rpbh_rotate_activations(self.x, self.perm, self.signs, out=self.xr)),
-            ("rpbh_dequantize", 1, lambda: o.rpbh_dequantize_weight(self.packed, self.norms, self.rows, self.d,
-                                                                    self.bits, self.cb, out_dtype=torch.bfloat16,
-                                                                    out=self.wq)),
-        ]
+
+        def rot(k):
+            o.rpbh_rotate_activations(self.xs[k % self.XSETS], self.perm, self.signs, out=self.xr)
+
+        def deq(k):
+            p = (k + 1) % self.PSETS
+            o.rpbh_dequantize_weight(self.packeds[p], self.normss[p], self.rows, self.d, self.bits, self.cb,
+                                     out_dtype=torch.bfloat16, out=self.wq)
+
+        return [("rpbh_quantize", 1, self._quantize), ("rpbh_rotate", 1, rot), ("rpbh_dequantize", 1, deq)]
 
     step = KVWorkload.step
 
@@ -374,9 +419,13 @@ class RPBHWorkload:
         self.d2h = sum(t.numel() * t.element_size() for t in self.pin_out)
 
     def e2e_step(self):
+        o = self.ops
         self.w.copy_(self.pin_in[0], non_blocking=True)
         self.x.copy_(self.pin_in[1], non_blocking=True)
-        self.step()
+        o.rpbh_quantize_weight(self.w, self.perm, self.signs, self.bits, self.cb, self.packed, self.norms)
+        o.rpbh_rotate_activations(self.x, self.perm, self.signs, out=self.xr)
+        o.rpbh_dequantize_weight(self.packed, self.norms, self.rows, self.d, self.bits, self.cb,
+                                 out_dtype=torch.bfloat16, out=self.wq)
         self.pin_out[0].copy_(self.wq, non_blocking=True)
         self.pin_out[1].copy_(self.xr, non_blocking=True)
 
@@ -448,22 +497,24 @@ def run_ours(args):
     # whole region. Event-record nodes between kernels would add several microseconds to each
     # kernel, so per-kernel durations come from a second timed region below: one graph per kernel
     # of back-to-back launches on the same buffers, bracketed by events.
-    wl.step()
+    wl.step(0)
     torch.cuda.synchronize()
     CHUNK = 500
 
-    def capture(fns, n):
+    def capture(fns, n, k0=0):
+        """A graph of n consecutive steps (or launches) k0 .. k0 + n - 1."""
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for _ in range(n):
+            for i in range(n):
                 for fn in fns:
-                    fn()
+                    fn(k0 + i)
         return g
 
     step_fns = [fn for _, _, fn in parts]
     warm = capture(step_fns, args.warmup)
     sizes = [CHUNK] * (args.steps // CHUNK) + ([args.steps % CHUNK] if args.steps % CHUNK else [])
-    chunks = [capture(step_fns, n) for n in sizes]
+    # the graphs continue the step index (which picks the rotating buffers) from one to the next
+    chunks = [capture(step_fns, n, args.warmup + sum(sizes[:c])) for c, n in enumerate(sizes)]
     warm.replay()
     torch.cuda.synchronize()
     barrier(world)
@@ -486,9 +537,11 @@ def run_ours(args):
     value = world * wl.units * args.steps / (ms_total / 1e3)
     del warm, chunks
 
-    # per-kernel durations (second timed region, same buffers)
+    # per-kernel durations (second timed region, same buffers): a whole number of buffer rotations,
+    # so that the warm-up replay and the timed one continue the same periodic sequence
     per_kernel = {}
-    reps = max(3, min(args.steps, 200))
+    rot = getattr(wl, "rotation", 1)
+    reps = max(rot, (max(3, min(args.steps, 200)) // rot) * rot)
     for name, n, fn in parts:
         g = capture([fn], reps)
         g.replay()
@@ -509,11 +562,10 @@ def run_ours(args):
     # kernels reported beside the step (same inputs, timed the same way, not part of `value`)
     beside = {}
     for name, n, fn in (wl.extras() if hasattr(wl, "extras") else []):
-        reps = max(3, min(args.steps, 200))
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for _ in range(reps):
-                fn()
+            for i in range(reps):
+                fn(i)
         g.replay()  # warm-up
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
@@ -555,8 +607,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": wl.name, "units_per_step_per_gpu": wl.units,
-                       "io_dtype": "bf16", "l2": "inputs larger than L2; no kernel reads data written by "
-                       "the kernel just before it", "launch": "CUDA graphs of up to 500 consecutive steps; per-kernel times from graphs of 200 back-to-back launches",
+                       "io_dtype": "bf16", "l2": wl.l2, "launch": f"CUDA graphs of up to 500 consecutive steps; per-kernel times from graphs of {reps} back-to-back launches",
                        "parallelism": f"replicas x{world} (no collective)"},
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
