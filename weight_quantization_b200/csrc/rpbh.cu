@@ -343,6 +343,8 @@ extern "C" wq_status rpbh_dequantize_weight(const uint8_t *packed, const void *r
     if (unrotate && rpbh_fast::supported(d, 1, dtype_size(out_dtype)) && aligned(perm, 16) && aligned(signs, 16))
         return rpbh_fast::dequantize_unrotate(packed, row_norms, norm_dtype, rows, d, bits, codebook, perm, signs, out,
                                               out_dtype, s);
+    if (!unrotate && aligned(packed, 16) && rpbh_fast::dequantize_rotated_fits(d, bits))
+        return rpbh_fast::dequantize_rotated(packed, row_norms, norm_dtype, rows, d, bits, codebook, out, out_dtype, s);
     rpbh::Codebook cb = {};
     for (int k = 0; k < (1 << bits); ++k) cb.c[k] = codebook[k];
     const int di = (int)d;

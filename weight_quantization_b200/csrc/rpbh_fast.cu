@@ -1027,6 +1027,96 @@ __global__ void __launch_bounds__(32 * kRotWarps, 2)
 }
 
 // ---------------------------------------------------------------------------------------------
+// rpbh_dequantize_weight without unrotate (_dequantize_rotated), persistent: each CTA walks rows
+// blockIdx.x, blockIdx.x + gridDim.x, ...; a row's codes (d/8 * bits bytes, a multiple of 16) come
+// in by 1-D bulk copy two rows ahead into one of two buffers, and its norm one row ahead into a
+// register, so no thread waits for memory in the middle of a row. Group g of 8 codes (bits
+// bytes, MSB first) gives 8 outputs, stored 16 bytes at a time.
+// ---------------------------------------------------------------------------------------------
+template <bool kNormBf16, bool kOutBf16, int BITS>
+__global__ void __launch_bounds__(256)
+    deq_rot_persistent(const uint8_t *__restrict__ packed, const void *__restrict__ row_norms, int rows, int d,
+                       Codebook cb, void *__restrict__ out) {
+    extern __shared__ unsigned char smem_raw[];
+    __shared__ float cbs[16];
+    unsigned char *base = align16(smem_raw);
+    const uint32_t nbytes = (uint32_t)(d / 8 * BITS);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + 2 * nbytes);
+    constexpr int L = 1 << BITS;
+    constexpr uint32_t kMask = (1u << BITS) - 1u;
+    if (threadIdx.x < L) {
+        // codebook.to(dtype): the bf16 rotated output multiplies bf16-rounded operands
+        const float c = cb.c[threadIdx.x];
+        cbs[threadIdx.x] = kOutBf16 ? bf16_to_f32(f32_to_bf16(c)) : c;
+    }
+    auto norm_of = [&](int r) {
+        return kNormBf16 ? bf16_to_f32(static_cast<const uint16_t *>(row_norms)[r])
+                         : static_cast<const float *>(row_norms)[r];
+    };
+    int row = blockIdx.x;
+    uint32_t n_iss0 = 0u, n_iss1 = 0u;  // thread 0: row copies issued into each buffer
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        for (int b = 0; b < 2; ++b) {
+            const int r = row + b * (int)gridDim.x;
+            if (r < rows) {
+                mbar_expect_tx(&bar[b], nbytes);
+                bulk_load(base + b * nbytes, packed + (int64_t)r * nbytes, nbytes, &bar[b]);
+                if (b == 0) ++n_iss0; else ++n_iss1;
+            }
+        }
+    }
+    __syncthreads();
+    float rho_next = row < rows ? norm_of(row) : 0.0f;
+    bool fault = false;
+    for (int it = 0; row < rows; ++it, row += gridDim.x) {
+        const int cur = it & 1;
+        const float rho = rho_next;
+        if (row + (int)gridDim.x < rows) rho_next = norm_of(row + gridDim.x);
+        const float rho_op = kOutBf16 ? bf16_to_f32(f32_to_bf16(rho)) : rho;
+        if (!fault && !mbar_wait_bounded(&bar[cur], (it >> 1) & 1, kMaxPolls)) {
+            fault = true;
+            atomicOr(&g_fault, 2u);
+        }
+        const unsigned char *src = base + cur * nbytes;
+        for (int g = threadIdx.x; g < d / 8; g += blockDim.x) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int b = 0; b < BITS; ++b) word = (word << 8) | src[g * BITS + b];
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(cbs[(word >> (BITS * (7 - i))) & kMask], rho_op);
+            if (kOutBf16) {
+                st_stream16(static_cast<uint16_t *>(out) + (int64_t)row * d + 8 * g,
+                            make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                       pack_bf16x2(v[6], v[7])));
+            } else {
+                float *o = static_cast<float *>(out) + (int64_t)row * d + 8 * g;
+                st_stream16(o, make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                                          __float_as_uint(v[3])));
+                st_stream16(o + 4, make_uint4(__float_as_uint(v[4]), __float_as_uint(v[5]), __float_as_uint(v[6]),
+                                              __float_as_uint(v[7])));
+            }
+        }
+        // every thread has read this buffer: it takes the row after next
+        fence_proxy_async_smem();
+        __syncthreads();
+        const int r2 = row + 2 * (int)gridDim.x;
+        if (threadIdx.x == 0 && r2 < rows && !fault) {
+            mbar_expect_tx(&bar[cur], nbytes);
+            bulk_load(base + cur * nbytes, packed + (int64_t)r2 * nbytes, nbytes, &bar[cur]);
+            if (cur == 0) ++n_iss0; else ++n_iss1;
+        }
+    }
+    // a fault may leave row copies in flight: give the last one into each buffer a bounded chance
+    if (fault && threadIdx.x == 0) {
+        if (n_iss0 > 0) mbar_wait_bounded(&bar[0], (n_iss0 - 1) & 1u, kMaxPolls);
+        if (n_iss1 > 0) mbar_wait_bounded(&bar[1], (n_iss1 - 1) & 1u, kMaxPolls);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
 // host dispatch
 // ---------------------------------------------------------------------------------------------
 int log2_block(int64_t d) {
@@ -1306,6 +1396,48 @@ wq_status dequantize_unrotate(const uint8_t *packed, const void *row_norms, int 
         case 6: return deq_dt<6>(nb, ob, bits, packed, row_norms, rows, d, cb, perm, signs, out, s);
         default: return WQ_ERR_SHAPE;
     }
+}
+
+bool dequantize_rotated_fits(int64_t d, int bits) {
+    const int64_t nbytes = d / 8 * bits;
+    return d % 8 == 0 && nbytes % 16 == 0 && 2 * nbytes + 64 + 1024 <= (int64_t)smem_limit();
+}
+
+template <bool kNB, bool kOB, int BITS>
+wq_status deq_rot_launch(const uint8_t *packed, const void *row_norms, int64_t rows, int64_t d, const Codebook &cb,
+                         void *out, cudaStream_t s) {
+    auto k = deq_rot_persistent<kNB, kOB, BITS>;
+    const size_t smem = (size_t)(d / 8 * BITS) * 2 + 16 + 16;
+    const wq_status st = prep(k, smem);
+    if (st != WQ_OK) return st;
+    // 128 or 256 threads, whichever leaves fewer idle group slots in a row's last pass
+    const int64_t groups = d / 8;
+    const int64_t idle128 = (groups + 127) / 128 * 128 - groups, idle256 = (groups + 255) / 256 * 256 - groups;
+    const int threads = idle128 < idle256 ? 128 : 256;
+    k<<<persistent_grid(k, threads, smem, rows), threads, smem, s>>>(packed, row_norms, (int)rows, (int)d, cb, out);
+    return launch_status();
+}
+
+template <bool kNB, bool kOB>
+wq_status deq_rot_bits(int bits, const uint8_t *packed, const void *row_norms, int64_t rows, int64_t d,
+                       const Codebook &cb, void *out, cudaStream_t s) {
+    switch (bits) {
+        case 2: return deq_rot_launch<kNB, kOB, 2>(packed, row_norms, rows, d, cb, out, s);
+        case 3: return deq_rot_launch<kNB, kOB, 3>(packed, row_norms, rows, d, cb, out, s);
+        case 4: return deq_rot_launch<kNB, kOB, 4>(packed, row_norms, rows, d, cb, out, s);
+        default: return WQ_ERR_BITS;
+    }
+}
+
+wq_status dequantize_rotated(const uint8_t *packed, const void *row_norms, int norm_dtype, int64_t rows, int64_t d,
+                             int bits, const float *codebook, void *out, int out_dtype, cudaStream_t s) {
+    Codebook cb = {};
+    for (int k = 0; k < (1 << bits); ++k) cb.c[k] = codebook[k];
+    const bool nb = norm_dtype == WQ_BF16, ob = out_dtype == WQ_BF16;
+    if (nb) return ob ? deq_rot_bits<true, true>(bits, packed, row_norms, rows, d, cb, out, s)
+                      : deq_rot_bits<true, false>(bits, packed, row_norms, rows, d, cb, out, s);
+    return ob ? deq_rot_bits<false, true>(bits, packed, row_norms, rows, d, cb, out, s)
+              : deq_rot_bits<false, false>(bits, packed, row_norms, rows, d, cb, out, s);
 }
 
 unsigned int read_and_clear_fault() {

@@ -24,6 +24,12 @@ wq_status dequantize_unrotate(const uint8_t *packed, const void *row_norms, int 
                               int bits, const float *codebook, const int32_t *perm, const int8_t *signs, void *out,
                               int out_dtype, cudaStream_t s);
 
+// _dequantize_rotated for rows whose codes (d/8 * bits bytes) are a multiple of 16 bytes and fit
+// twice in shared memory: a persistent kernel that fetches each row's codes ahead by bulk copy.
+bool dequantize_rotated_fits(int64_t d, int bits);
+wq_status dequantize_rotated(const uint8_t *packed, const void *row_norms, int norm_dtype, int64_t rows, int64_t d,
+                             int bits, const float *codebook, void *out, int out_dtype, cudaStream_t s);
+
 // Reads and clears the fault bits of these kernels (bit 1: a bounded wait for a row copy ran out).
 unsigned int read_and_clear_fault();
 
