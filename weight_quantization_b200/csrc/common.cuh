@@ -186,6 +186,12 @@ __device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap *map, int x,
                  "r"(x), "r"(y), "r"(smem_u32(src)), "l"(pol)
                  : "memory");
 }
+// Hint: bring `bytes` (a multiple of 16, the address 16-byte aligned, all inside one allocation)
+// of global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until at most N committed bulk groups still read their shared-memory source.
 template <int N>

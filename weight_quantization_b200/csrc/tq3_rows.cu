@@ -372,6 +372,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
     const float post = tq3::fwht_post();
 
     int64_t tile = blockIdx.x;
+    const bool pf_ok = ((reinterpret_cast<uintptr_t>(packed) | reinterpret_cast<uintptr_t>(norms) |
+                         reinterpret_cast<uintptr_t>(scales)) & 15) == 0;
     pdl_wait();  // the records may come from the kernel before this one
     Rec cur = load_rec(packed, norms, scales, n_vec, tile * kTile + tid);
     for (int it = 0; tile < n_tiles; ++it, tile += gridDim.x) {
@@ -379,6 +381,17 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         // overlaps this kernel's tail (it still waits for this kernel to finish before reading)
         if (tile + gridDim.x >= n_tiles) pdl_trigger();
         const Rec nxt = load_rec(packed, norms, scales, n_vec, (tile + gridDim.x) * kTile + tid);
+        // the records of the tile after that go into L2 now, so next iteration's load finds them
+        // there (whole 16-byte units inside the arrays only)
+        if (tid == 0 && pf_ok && tile + 2 * gridDim.x < n_tiles) {
+            const int64_t v0 = (tile + 2 * gridDim.x) * kTile;
+            const int64_t cnt = (n_vec - v0 < kTile ? n_vec - v0 : kTile) & ~int64_t(3);
+            if (cnt > 0) {
+                bulk_prefetch_l2(packed + v0 * 48, (uint32_t)(cnt * 48));
+                bulk_prefetch_l2(norms + v0, (uint32_t)(cnt * 4));
+                bulk_prefetch_l2(scales + v0, (uint32_t)(cnt * 4));
+            }
+        }
         unsigned char *buf = obuf + (it % G::kBufs) * G::kTileBytes;
         if (tid == 0) bulk_wait_read<G::kBufs - 1>();  // the store that last read this buffer is done
         __syncthreads();
