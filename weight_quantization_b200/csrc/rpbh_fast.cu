@@ -748,15 +748,18 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
 // sums alternate between two sets by row, so a set is rewritten only after the barrier between.
 // A timed-out wait sets the fault flag but ends no thread's loop early, so every thread meets
 // every barrier.
-template <int B, bool kBf16, int BITS, bool kSym>
-__global__ void __launch_bounds__(kMaxThreads, 2)
+// kSlotsT = 1: the form for rows with at most one block group per warp (h = 1024 rows of a few
+// blocks): one register slot per lane, so more CTAs fit an SM.
+template <int B, bool kBf16, int BITS, bool kSym, int kSlotsT = 0>
+__global__ void __launch_bounds__(kSlotsT == 1 ? 128 : kMaxThreads, kSlotsT == 1 ? 5 : 2)
     quantize_warp(const void *__restrict__ w, int rows, int d, float post, const int32_t *__restrict__ perm,
                   const int8_t *__restrict__ signs, Edges E, uint8_t *__restrict__ packed,
                   void *__restrict__ row_norms) {
     using G = Geo<B>;
     constexpr int S = G::S, H = G::H;
-    constexpr int kBpw = 32 / S;    // blocks a warp works on at once: lane = sub-block * S + row / column
-    constexpr int kSlots = 64 / S;  // register slots per lane (the host checks the warp's share fits)
+    constexpr int kBpw = 32 / S;  // blocks a warp works on at once: lane = sub-block * S + row / column
+    // register slots per lane (the host checks the warp's share fits)
+    constexpr int kSlots = kSlotsT ? kSlotsT : 64 / S;
     constexpr int esz = kBf16 ? 2 : 4;
     static_assert(S <= 32, "a block's rows must fit one warp");
     extern __shared__ unsigned char smem_raw[];
@@ -1264,6 +1267,21 @@ wq_status quantize_b(const void *w, int64_t rows, int64_t d, const int32_t *perm
     if constexpr (B == 5 || (B == 4 && kBf16)) {
         constexpr int64_t S = int64_t(1) << B;
         const int64_t groups = ((d >> (2 * B)) + 32 / S - 1) / (32 / S);
+        // at most one block group per warp: the one-slot form
+        if constexpr (B == 5) {
+            if ((!kSym || E.steps) && persistent_fits(d, kBf16 ? 2 : 4) && groups <= threads / 32 &&
+                threads <= 128) {
+                const size_t psmem = pers_smem(d, kBf16 ? 2 : 4);
+                auto kw = quantize_warp<B, kBf16, BITS, kSym, 1>;
+                st = prep(kw, psmem);
+                if (st != WQ_OK) return st;
+                if (blocks_per_sm(reinterpret_cast<const void *>(kw), threads, psmem) >= 1) {
+                    kw<<<persistent_grid(kw, threads, psmem, rows), threads, psmem, s>>>(
+                        w, (int)rows, (int)d, fwht_post(d & -d), perm, signs, E, packed, row_norms);
+                    return launch_status();
+                }
+            }
+        }
         if ((!kSym || E.steps) && persistent_fits(d, kBf16 ? 2 : 4) &&
             (groups + threads / 32 - 1) / (threads / 32) <= 64 / S) {
             const size_t psmem = pers_smem(d, kBf16 ? 2 : 4);
