@@ -49,6 +49,16 @@ def measured_peaks():
     return HBM_FALLBACK_GBS, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s measured on this machine (a cuBLAS burst), or the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    return 1590.0, "fallback"
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons, sampled every 200 ms while the timed region runs."""
 
@@ -445,11 +455,97 @@ class RPBHWorkload:
         return done * self.d / dt, f"first {done} weight rows quantized + dequantized (no activations), {dt:.1f} s"
 
 
+class RPBHLinearWorkload:
+    """The fused RPBH linear layer of forward on the LLM MLP shape: y[2048, 4096] = x_rot W'^T + b,
+    W'[4096, 11008] held as 3-bit codes and row norms (from quantizing the LLM weight), x_rot bf16."""
+
+    metric = "RPBH fused dequantize + linear FLOP/s (2 m n d per call)"
+    unit = "FLOP/s"
+    bound = "tensor"
+
+    def __init__(self, dev, out_f=4096, d=11008, m=2048, bits=3, seed=5):
+        from weight_quantization_b200 import ops
+        self.ops = ops
+        self.name = f"rpbh-linear-w{out_f}x{d}-x{m}-b{bits}"
+        self.out_f, self.d, self.m, self.bits = out_f, d, m, bits
+        bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        perm, signs = inputs.rpbh_params(d)
+        perm_d, signs_d = torch.from_numpy(perm).to(dev), torch.from_numpy(signs).to(dev)
+        w = bf(inputs.llm_weight(out_f, d, seed=seed)).to(dev)
+        self.cb = ops.rpbh_codebook(bits, d)
+        packed, norms = ops.rpbh_quantize_weight(w, perm_d, signs_d, bits, self.cb)
+        del w
+        x = bf(inputs.activations(m, d, seed=seed)).to(dev)
+        xr = ops.rpbh_rotate_activations(x, perm_d, signs_d)
+        # x_rot (45 MB) and the codes (17 MB) are smaller than L2: each rotates over copies
+        X, P = self.XSETS, self.PSETS
+        self.xs = [xr.clone() for _ in range(X)]
+        self.packeds = [packed.clone() for _ in range(P)]
+        self.norms = norms
+        self.bias = (torch.randn(out_f, generator=torch.Generator().manual_seed(seed)) * 0.01).to(torch.bfloat16).to(dev)
+        self.y = torch.empty(m, out_f, dtype=torch.bfloat16, device=dev)
+        self.host_x = xr.cpu()
+        self.units = 2 * m * out_f * d
+        self.kernels = ["rpbh_linear"]
+        self.flops_per_launch = {"rpbh_linear": 2 * m * out_f * d}
+        self.bytes_per_launch = {"rpbh_linear": packed.numel() + 2 * out_f + 2 * m * d + 2 * m * out_f + 2 * out_f}
+        self.l2 = (f"x_rot rotates over {X} copies and the codes over {P} sets: launch k uses x_rot copy "
+                   f"k % {X} and code set k % {P}")
+
+    XSETS, PSETS = 4, 3
+    rotation = 12
+
+    def _linear(self, k, x=None):
+        self.ops.rpbh_linear(self.packeds[k % self.PSETS], self.norms, self.out_f, self.d, self.bits, self.cb,
+                             self.xs[k % self.XSETS] if x is None else x, bias=self.bias, out=self.y)
+
+    def parts(self):
+        return [("rpbh_linear", 1, self._linear)]
+
+    def extras(self):
+        return []
+
+    step = KVWorkload.step
+
+    def e2e_setup(self):
+        self.pin_in = self.host_x.pin_memory()
+        self.pin_out = torch.empty(self.m, self.out_f, dtype=torch.bfloat16).pin_memory()
+        self.h2d = self.pin_in.numel() * 2
+        self.d2h = self.pin_out.numel() * 2
+
+    def e2e_step(self):
+        """x_rot in from pinned memory, the layer through the public call, y out (the weight codes
+        stay resident, as in serving)."""
+        self.xs[0].copy_(self.pin_in, non_blocking=True)
+        self._linear(0)
+        self.pin_out.copy_(self.y, non_blocking=True)
+
+    def oracle_rate(self, budget_s=10.0):
+        import oracle
+        oracle.lib()
+        p = self.packeds[0].cpu().numpy()
+        n32 = self.norms.float().cpu().numpy()
+        x = self.host_x.view(torch.int16).numpy().view(np.uint16)
+        b = self.bias.cpu().view(torch.int16).numpy().view(np.uint16)
+        rows_w = 64  # output features per sample (whole rows of the packed stream)
+        row_bytes = self.d // 8 * self.bits
+        done, t0, flops = 0, time.perf_counter(), 0
+        while time.perf_counter() - t0 < budget_s and (done + 1) * rows_w <= self.out_f:
+            lo = done * rows_w
+            oracle.rpbh_linear(p[lo * row_bytes:(lo + rows_w) * row_bytes], n32[lo:lo + rows_w], rows_w, self.d,
+                               self.bits, self.cb, x[:64], b[lo:lo + rows_w])
+            flops += 2 * 64 * rows_w * self.d
+            done += 1
+        dt = time.perf_counter() - t0
+        return flops / dt, f"{done} blocks of 64 output features x 64 activation rows (dequantize + fp64 product), {dt:.1f} s"
+
+
 WORKLOADS = {
     "kv": KVWorkload,
     "longctx": LongContextWorkload,
     "rpbh-llm": lambda dev: RPBHWorkload(dev),
     "rpbh-dit": lambda dev: RPBHWorkload(dev, rows=12288, d=3072, xrows=4096, bits=3, seed=4),
+    "rpbh-linear": RPBHLinearWorkload,
 }
 
 
@@ -601,6 +697,17 @@ def run_ours(args):
         rate, sample = wl.oracle_rate(args.cpu_seconds)
         cpu = {"value": rate, "unit": wl.unit, "cores": 1, "kind": "oracle", "sample": sample}
 
+    if getattr(wl, "bound", "hbm") == "tensor":
+        tpeak, tkind = measured_tensor_peak()
+        tflops = wl.flops_per_launch[dom] / (per_kernel[dom]["avg_us"] * 1e-6) / 1e12
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": tflops, "peak": tpeak, "peak_kind": tkind,
+                    "unit": "TFLOP/s", "frac": tflops / tpeak, "traffic": traffic_bytes(dom),
+                    "algorithmic_flops_per_launch": wl.flops_per_launch[dom],
+                    "algorithmic_bytes_per_launch": wl.bytes_per_launch[dom]}
+    else:
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                    "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_bytes(dom),
+                    "algorithmic_bytes_per_launch": wl.bytes_per_launch[dom]}
     if rank == 0:
         line = {
             "metric": wl.metric, "value": value, "unit": wl.unit, "n_gpus": world, "steps": args.steps,
@@ -609,10 +716,7 @@ def run_ours(args):
             "config": {"workload": wl.name, "units_per_step_per_gpu": wl.units,
                        "io_dtype": "bf16", "l2": wl.l2, "launch": f"CUDA graphs of up to 500 consecutive steps; per-kernel times from graphs of {reps} back-to-back launches",
                        "parallelism": f"replicas x{world} (no collective)"},
-            "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": traffic_bytes(dom),
-                         "algorithmic_bytes_per_launch": wl.bytes_per_launch[dom]},
+            "roofline": roofline,
             "kernels": per_kernel,
             **({"kernels_beside_step": beside} if beside else {}),
             "e2e": {"value": e2e_value, "unit": wl.unit, "h2d_bytes_per_step": wl.h2d,

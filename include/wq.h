@@ -156,6 +156,24 @@ wq_status rpbh_rotate_activations(const void *x, int dtype, int64_t rows, int64_
                                   const int32_t *perm, const int8_t *signs, void *x_rot,
                                   void *stream);
 
+/* rpbh_linear -- the linear layer of OrbitQuantizer.forward on the rotated activations,
+ * y = F.linear(x_rot, W', bias) with W' the rotated-basis dequantized weight (as
+ * rpbh_dequantize_weight with unrotate = 0 and bf16 output), without writing W' out: the codes
+ * are unpacked into the tensor-core operand on chip. y[i][n] = bf16(sum_k x_rot[i][k] *
+ * bf16(codebook[code[n][k]]) * bf16(row_norm[n]) + bias[n]), the sum in fp32 on the tensor cores;
+ * the row norm scales the sum instead of each product, so y agrees with the product of the bf16
+ * W' to within 2^-8 relative per term (plus fp32 summation and the final bf16 rounding).
+ *   packed     device, as written by rpbh_quantize_weight for out_features x d, 16-byte aligned.
+ *   row_norms  device, out_features entries of norm_dtype.  codebook  host, 2^bits fp32.
+ *   x_rot      device, m x d bf16 (rpbh_rotate_activations output), 16-byte aligned.
+ *   bias       device, out_features bf16, or NULL for none.
+ *   y          device, m x out_features bf16 (row-major), 2-byte aligned.
+ * d must be a multiple of 64. Errors: WQ_ERR_NULL, WQ_ERR_SHAPE (negative sizes, d not a
+ * multiple of 64 or above 2^20), WQ_ERR_BITS, WQ_ERR_DTYPE, WQ_ERR_ALIGN, WQ_ERR_CUDA. */
+wq_status rpbh_linear(const uint8_t *packed, const void *row_norms, int norm_dtype,
+                      int64_t out_features, int64_t d, int bits, const float *codebook,
+                      const void *x_rot, int64_t m, const void *bias, void *y, void *stream);
+
 /* rpbh_packed_bytes -- size of the packed bitstream: ceil(rows * d / 8) * bits (-1 on a bad
  * argument). */
 int64_t rpbh_packed_bytes(int64_t rows, int64_t d, int bits);
@@ -179,7 +197,8 @@ wq_status wq_rpbh_codebook(int bits, int64_t d, float *out);
 /* wq_device_fault -- reads and clears the library's sticky device fault bits. A kernel whose
  * bounded wait runs out (which does not happen in normal operation) sets a bit and returns early,
  * leaving its outputs unspecified: bit 0 a TQ3 kernel waiting for a TMA tile, bit 1 an RPBH kernel
- * waiting for a row copy, bit 3 the tensor-core TQ3 encoder waiting for a tile or its product.
+ * waiting for a row copy, bit 3 the tensor-core TQ3 encoder waiting for a tile or its product,
+ * bit 4 rpbh_linear waiting for a tile, the unpacked weights or its product.
  * Synchronous (a device-to-host copy on the legacy default stream); `flags` is host memory.
  * Errors: WQ_ERR_NULL, WQ_ERR_CUDA. */
 wq_status wq_device_fault(unsigned int *flags);

@@ -253,6 +253,21 @@ def rpbh_dequantize_rotated(packed, row_norms_f32, rows, d, bits, codebook, out_
     return out
 
 
+def rpbh_linear(packed, row_norms_f32, out_features, d, bits, codebook, x_rot_bits, bias_bits=None):
+    """Page "orbit_quant.py", forward: F.linear(x_rot, W', bias) with W' the rotated-basis weight in
+    bf16 (_dequantize_rotated in the weight dtype, as rpbh_dequantize_rotated(out_bf16=True)).
+    The product is taken in fp64 (a library matmul). Returns (y, abs_sum): y [m, out_features] and
+    abs_sum[i][n] = sum_k |x_rot[i][k] W'[n][k]|, which bounds the rounding of any fp32 evaluation."""
+    wq = bf16_array_to_f32(rpbh_dequantize_rotated(packed, row_norms_f32, out_features, d, bits, codebook,
+                                                   out_bf16=True)).astype(np.float64)
+    x = bf16_array_to_f32(np.asarray(x_rot_bits, np.uint16)).astype(np.float64)
+    y = x @ wq.T
+    a = np.abs(x) @ np.abs(wq).T
+    if bias_bits is not None:
+        y = y + bf16_array_to_f32(np.asarray(bias_bits, np.uint16)).astype(np.float64)[None, :]
+    return y, a
+
+
 def rpbh_dequantize(packed, row_norms_f32, rows, d, bits, codebook, inv_perm, signs, h):
     out = np.zeros((rows, d), np.float32)
     lib().or_rpbh_dequantize(_p(_c(packed, np.uint8)), _p(_c(row_norms_f32, np.float32)), rows, d, bits,

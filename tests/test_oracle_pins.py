@@ -468,6 +468,29 @@ def test_rpbh_dequantize_matches_dense(oracle):
     assert np.abs(w - wrot.astype(np.float64) @ R).max() < 1e-5
 
 
+def test_rpbh_linear_one_hot_and_zero_inputs(oracle):
+    """forward's F.linear on the rotated activations: a one-hot activation row e_k returns column k
+    of the bf16 rotated weight plus the bias (so the product is x W'^T, not a transpose of it), and
+    zero activations return the bias exactly."""
+    out_f, d, bits = 5, 64, 3
+    cb = oracle.rpbh_codebook(bits, d)
+    codes = inputs.uniform_int((out_f, d), 8, seed=72)
+    packed = oracle.pack_codes(codes, bits)
+    norms = (np.abs(inputs.gaussian((out_f,), seed=73)) + 0.1).astype(np.float32)
+    bias = oracle.f32_array_to_bf16(inputs.gaussian((out_f,), seed=74).astype(np.float32))
+    one = oracle.f32_array_to_bf16(np.eye(d, dtype=np.float32))
+    y, a = oracle.rpbh_linear(packed, norms, out_f, d, bits, cb, one, bias)
+    w16 = oracle.bf16_array_to_f32(oracle.rpbh_dequantize_rotated(packed, norms, out_f, d, bits, cb, out_bf16=True))
+    b32 = oracle.bf16_array_to_f32(bias)
+    assert y.shape == (d, out_f)
+    assert np.array_equal(y, w16.T.astype(np.float64) + b32[None, :].astype(np.float64))
+    assert np.array_equal(a, np.abs(w16.T).astype(np.float64))
+    zero = np.zeros((3, d), np.uint16)
+    y0, a0 = oracle.rpbh_linear(packed, norms, out_f, d, bits, cb, zero, bias)
+    assert np.array_equal(y0, np.broadcast_to(b32.astype(np.float64), (3, out_f)))
+    assert not a0.any()
+
+
 def test_rpbh_rotate_bf16_matches_dense(oracle):
     d = 640
     perm, signs = inputs.rpbh_params(d)

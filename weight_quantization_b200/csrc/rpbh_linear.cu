@@ -1,0 +1,294 @@
+// Fused RPBH linear layer on sm_100a: page "orbit_quant.py", forward (x_rot = rpbh_forward(x),
+// then F.linear(x_rot, W', bias)), with W' the rotated-basis dequantized weight
+// (_dequantize_rotated: codebook[codes] * norms in the weight dtype). W' is never written out: its
+// packed codes are unpacked straight into the tensor-core operand in shared memory.
+//
+// One CTA computes a 128 x 256 tile of D = W'_tile x_rot_tile^T (128 output features = the
+// product's M and the accumulator's lanes, 256 activation rows = N and its columns), K = d in
+// chunks of 64 (one 128-byte swizzle atom of bf16):
+//   * warp 0, lane 0: TMA loads of x_rot [256 x 64] bf16 tiles (128-byte swizzle) into a ring of
+//     four stages, and the products: four tcgen05.mma.kind::f16 (M = 128, N = 256, K = 16) per
+//     chunk, accumulating in 256 tensor-memory columns, each chunk's commit releasing its stage;
+//   * warps 4..7: thread p owns output feature n0 + p: it loads the chunk's 8 * bits code bytes
+//     of its row, unpacks the 64 codes (MSB-first stream, pack_codes) and looks each up in the
+//     codebook rounded to bf16 (a shuffle: lane l holds centroid l mod 2^bits), writing the 128-byte
+//     row of the operand tile with the 128-byte swizzle; then, after the last product, the
+//     epilogue: accumulator row p, column j is y[m0 + j][n0 + p] / rho, so
+//     y = bf16(acc * bf16(rho_n) + bias_n), stored so that a warp writes 32 consecutive features.
+// The row norm is applied to the accumulated sum instead of to every element: the standalone
+// dequantizer rounds bf16(codebook) * bf16(rho) to bf16 per element, this kernel does not, so
+// the two differ by at most 2^-8 relative per term (the tolerance the tests use).
+// Every wait is bounded; a timeout sets the fault flag, after which no wait or issue happens
+// and the kernel runs out, results void.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <climits>
+#include <cstring>
+
+#include "common.cuh"
+#include "tcgen05.cuh"
+#include "rpbh_linear.cuh"
+#include "wq.h"
+
+namespace wq {
+namespace rpbh_linear {
+
+constexpr int kTM = 128;  // output features per tile
+constexpr int kTN = 256;  // activation rows per tile
+constexpr int kTK = 64;   // K per chunk
+constexpr int kStages = 4;
+constexpr int kThreads = 256;
+constexpr int kABytes = kTM * kTK * 2;
+constexpr int kBBytes = kTN * kTK * 2;
+constexpr int kOffA = 0;
+constexpr int kOffB = kStages * kABytes;
+constexpr int kOffBar = kOffB + kStages * kBBytes;  // full_a[4], full_b[4], empty[4], done, then the TMEM address
+constexpr int kSmem = 1024 + kOffBar + 8 * (3 * kStages + 1) + 16;
+static_assert(kSmem <= 232448, "the ring must fit the 227 KB a CTA may use");
+// fp32 accumulator, bf16 A and B, both K-major, N = 256, M = 128
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTN >> 3) << 17) |
+                            ((uint32_t)(kTM >> 4) << 24);
+constexpr uint32_t kMaxPolls = 1u << 24;
+
+__device__ unsigned int g_fault;
+
+struct CodebookBf16 {
+    uint16_t c[16];  // the codebook rounded to bf16 (codebook.to(dtype))
+};
+
+__device__ __forceinline__ unsigned char *align1024(unsigned char *p) {
+    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Code i (0 .. 63) of a chunk whose 8 * BITS bytes are held as big-endian 32-bit words W
+// (stream bit b is bit 31 - b % 32 of W[b / 32]).
+template <int BITS>
+__device__ __forceinline__ uint32_t code_at(const uint32_t (&W)[2 * BITS], int i) {
+    const int o = BITS * i, q = o >> 5, r = o & 31;
+    constexpr uint32_t kMask = (1u << BITS) - 1u;
+    if (r + BITS <= 32) return (W[q] >> (32 - r - BITS)) & kMask;
+    return __funnelshift_l(W[q + 1], W[q], r + BITS - 32) & kMask;
+}
+
+template <int BITS, bool kNormBf16>
+__global__ void __launch_bounds__(kThreads, 1)
+    linear_kernel(const uint8_t *__restrict__ packed, const void *__restrict__ row_norms, int out_f, int d,
+                  const __grid_constant__ CUtensorMap xmap, int m_rows, const uint16_t *__restrict__ bias,
+                  CodebookBf16 cb, uint16_t *__restrict__ y) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *const base = align1024(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * kTM, m0 = blockIdx.y * kTN;
+    const int nchunks = d / kTK;
+    uint64_t *const full_a = reinterpret_cast<uint64_t *>(base + kOffBar);  // the 4 unpacking warps arrive
+    uint64_t *const full_b = full_a + kStages;                             // the TMA of x_rot lands
+    uint64_t *const empty = full_b + kStages;                              // the chunk's products are done
+    uint64_t *const done = empty + kStages;                                // every product is done
+    uint32_t *const tslot = reinterpret_cast<uint32_t *>(done + 1);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full_a[s], 4);
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(done, 1);
+    }
+    if (warp == 0) tmem_alloc(tslot, kTN);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot;
+    bool fault = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            uint32_t issued[kStages] = {0u, 0u, 0u, 0u};  // x_rot copies issued per stage (fault path)
+            auto load_b = [&](int c) {
+                const int s = c % kStages;
+                mbar_expect_tx(&full_b[s], kBBytes);
+                tma_load_2d(base + kOffB + s * kBBytes, &xmap, c * kTK, m0, &full_b[s]);
+                ++issued[s];
+            };
+            for (int c = 0; c < kStages && c < nchunks; ++c) load_b(c);
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % kStages;
+                const uint32_t ph = (uint32_t)(c / kStages) & 1u;
+                if (!mbar_wait_bounded(&full_b[s], ph, kMaxPolls) || !mbar_wait_bounded(&full_a[s], ph, kMaxPolls)) {
+                    fault = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t ad = sw128_desc(smem_u32(base + kOffA + s * kABytes));
+                const uint64_t bd = sw128_desc(smem_u32(base + kOffB + s * kBBytes));
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // K = 16 per instruction: 32 bytes into each 128-byte row
+                    mma_bf16(tmem, ad + (uint32_t)(ks * 2), bd + (uint32_t)(ks * 2), kIdesc, (c > 0 || ks > 0) ? 1u : 0u);
+                mma_commit(&empty[s]);
+                // the previous chunk's stage takes the chunk kStages after it once its products are done
+                if (c >= 1 && c - 1 + kStages < nchunks) {
+                    const int sp = (c - 1) % kStages;
+                    if (!mbar_wait_bounded(&empty[sp], (uint32_t)((c - 1) / kStages) & 1u, kMaxPolls)) {
+                        fault = true;
+                        break;
+                    }
+                    load_b(c - 1 + kStages);
+                }
+            }
+            mma_commit(done);  // arrives once every product issued above is done
+            if (fault) {
+                // give the copies still in flight a bounded chance to land before the memory goes away
+                for (int s = 0; s < kStages; ++s)
+                    if (issued[s] > 0) mbar_wait_bounded(&full_b[s], (issued[s] - 1) & 1u, kMaxPolls);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        const int p = threadIdx.x - 128;  // this thread's output feature within the tile (accumulator lane)
+        const int n = n0 + p;
+        const bool valid = n < out_f;
+        const uint8_t *const src = packed + (int64_t)(valid ? n : 0) * (d / 8 * BITS);
+        // lane l holds the bf16 centroid l mod 2^bits: a shuffle from the lane named by a code is the lookup
+        const uint32_t cbv = cb.c[lane & ((1 << BITS) - 1)];
+        unsigned char *const rowA = base + kOffA + p * 128;
+        const int sw = p & 7;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % kStages;
+            if (c >= kStages && !fault) {
+                bool ok = true;
+                if (lane == 0) ok = mbar_wait_bounded(&empty[s], (uint32_t)(c / kStages - 1) & 1u, kMaxPolls);
+                if (!__all_sync(0xffffffffu, ok)) fault = true;
+            }
+            // the chunk's 8 * BITS code bytes, as big-endian words
+            uint32_t W[2 * BITS];
+#pragma unroll
+            for (int q = 0; q < BITS; ++q) {
+                const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src + c * 8 * BITS) + q);
+                W[2 * q] = __byte_perm(v.x, 0u, 0x0123);
+                W[2 * q + 1] = __byte_perm(v.y, 0u, 0x0123);
+            }
+            unsigned char *const A = rowA + s * kABytes;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {  // 16-byte chunk j: k = 8j .. 8j + 7
+                uint32_t w4[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t lo = __shfl_sync(0xffffffffu, cbv, (int)code_at<BITS>(W, 8 * j + 2 * u));
+                    const uint32_t hi = __shfl_sync(0xffffffffu, cbv, (int)code_at<BITS>(W, 8 * j + 2 * u + 1));
+                    w4[u] = valid ? (lo | (hi << 16)) : 0u;
+                }
+                *reinterpret_cast<uint4 *>(A + ((j ^ sw) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            fence_proxy_async_smem();  // written by threads, read by the tensor core
+            __syncwarp();
+            if (lane == 0 && !fault) mbar_arrive(&full_a[s]);
+        }
+        // epilogue: y[m][n] = bf16(acc[p][m - m0] * bf16(rho_n) + bias_n)
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait_bounded(done, 0u, kMaxPolls);
+        if (!__all_sync(0xffffffffu, ok)) fault = true;
+        tc_fence_after();
+        float rho = 0.0f, b = 0.0f;
+        if (valid) {
+            rho = kNormBf16 ? bf16_to_f32(static_cast<const uint16_t *>(row_norms)[n])
+                            : static_cast<const float *>(row_norms)[n];
+            rho = bf16_to_f32(f32_to_bf16(rho));
+            if (bias) b = bf16_to_f32(bias[n]);
+        }
+        const uint32_t lanes = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+#pragma unroll 1
+        for (int j = 0; j < kTN / 32; ++j) {
+            float v[32];
+            tmem_ld32(lanes + 32u * j, v);
+            tmem_wait(v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int m = m0 + 32 * j + i;
+                if (valid && m < m_rows) y[(int64_t)m * out_f + n] = f32_to_bf16(__fmaf_rn(v[i], rho, b));
+            }
+        }
+    }
+    if (fault && (lane == 0)) atomicOr(&g_fault, 16u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTN);
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------------
+namespace {
+// fp32 -> bf16, round to nearest even (the codebook's .to(dtype)); the codebook is finite
+uint16_t bf16_rne(float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+template <int BITS, bool kNB>
+wq_status launch(const uint8_t *packed, const void *row_norms, int64_t out_f, int64_t d, const CUtensorMap &xm,
+                 int64_t m, const uint16_t *bias, const CodebookBf16 &cb, uint16_t *y, cudaStream_t s) {
+    auto k = linear_kernel<BITS, kNB>;
+    if (!ensure_dynamic_smem(reinterpret_cast<const void *>(k), kSmem)) return WQ_ERR_CUDA;
+    const dim3 grid((unsigned)((out_f + kTM - 1) / kTM), (unsigned)((m + kTN - 1) / kTN));
+    k<<<grid, kThreads, kSmem, s>>>(packed, row_norms, (int)out_f, (int)d, xm, (int)m, bias, cb, y);
+    return launch_status();
+}
+
+template <bool kNB>
+wq_status by_bits(int bits, const uint8_t *packed, const void *row_norms, int64_t out_f, int64_t d,
+                  const CUtensorMap &xm, int64_t m, const uint16_t *bias, const CodebookBf16 &cb, uint16_t *y,
+                  cudaStream_t s) {
+    switch (bits) {
+        case 2: return launch<2, kNB>(packed, row_norms, out_f, d, xm, m, bias, cb, y, s);
+        case 3: return launch<3, kNB>(packed, row_norms, out_f, d, xm, m, bias, cb, y, s);
+        case 4: return launch<4, kNB>(packed, row_norms, out_f, d, xm, m, bias, cb, y, s);
+        default: return WQ_ERR_BITS;
+    }
+}
+}  // namespace
+
+unsigned int read_and_clear_fault() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_fault, sizeof v) != cudaSuccess) return 0x80000000u;
+    if (v) cudaMemcpyToSymbol(g_fault, &zero, sizeof zero);
+    return v;
+}
+
+}  // namespace rpbh_linear
+}  // namespace wq
+
+using namespace wq;
+
+extern "C" wq_status rpbh_linear(const uint8_t *packed, const void *row_norms, int norm_dtype, int64_t out_features,
+                                 int64_t d, int bits, const float *codebook, const void *x_rot, int64_t m,
+                                 const void *bias, void *y, void *stream) {
+    if (out_features < 0 || d < 0 || m < 0) return WQ_ERR_SHAPE;
+    if (bits < 2 || bits > 4) return WQ_ERR_BITS;
+    if (norm_dtype != WQ_F32 && norm_dtype != WQ_BF16) return WQ_ERR_DTYPE;
+    if (d % 64 != 0 || d > (int64_t)1 << 20 || out_features > INT32_MAX / 2 || m > INT32_MAX / 2) return WQ_ERR_SHAPE;
+    if (out_features == 0 || m == 0) return WQ_OK;
+    if (d == 0) return WQ_ERR_SHAPE;
+    if (!packed || !row_norms || !codebook || !x_rot || !y) return WQ_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(packed) & 15) || (reinterpret_cast<uintptr_t>(x_rot) & 15) ||
+        (reinterpret_cast<uintptr_t>(y) & 1) || (reinterpret_cast<uintptr_t>(bias) & 1) ||
+        (reinterpret_cast<uintptr_t>(row_norms) & (norm_dtype == WQ_BF16 ? 1 : 3)))
+        return WQ_ERR_ALIGN;
+    rpbh_linear::CodebookBf16 cb = {};
+    for (int k = 0; k < (1 << bits); ++k) cb.c[k] = rpbh_linear::bf16_rne(codebook[k]);
+    CUtensorMap xm;
+    if (!make_tmap_2d(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_rot, (uint64_t)d, (uint64_t)m, (uint64_t)d * 2,
+                      rpbh_linear::kTK, rpbh_linear::kTN))
+        return WQ_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const auto *b = static_cast<const uint16_t *>(bias);
+    auto *yo = static_cast<uint16_t *>(y);
+    return norm_dtype == WQ_BF16
+               ? rpbh_linear::by_bits<true>(bits, packed, row_norms, out_features, d, xm, m, b, cb, yo, s)
+               : rpbh_linear::by_bits<false>(bits, packed, row_norms, out_features, d, xm, m, b, cb, yo, s);
+}

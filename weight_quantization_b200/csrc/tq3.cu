@@ -27,6 +27,7 @@
 #include "rpbh_fast.cuh"
 #include "tq3_common.cuh"
 #include "tq3_mma.cuh"
+#include "rpbh_linear.cuh"
 #include "tq3_rows.cuh"
 #include "wq.h"
 
@@ -486,7 +487,8 @@ extern "C" wq_status wq_device_fault(unsigned int *flags) {
     const unsigned int r = rpbh_fast::read_and_clear_fault();
     const unsigned int q = tq3_rows::read_and_clear_fault();
     const unsigned int t = tq3_mma::read_and_clear_fault();
-    if ((r | q | t) & 0x80000000u) return WQ_ERR_CUDA;
-    *flags = v | r | q | t;
+    const unsigned int l = rpbh_linear::read_and_clear_fault();
+    if ((r | q | t | l) & 0x80000000u) return WQ_ERR_CUDA;
+    *flags = v | r | q | t | l;
     return WQ_OK;
 }

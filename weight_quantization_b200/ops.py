@@ -29,6 +29,7 @@ PROTOTYPES = {
     "rpbh_quantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp]),
     "rpbh_dequantize_weight": (_int, [_vp, _vp, _int, _i64, _i64, _int, _vp, _vp, _vp, _int, _vp, _int, _vp]),
     "rpbh_rotate_activations": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "rpbh_linear": (_int, [_vp, _vp, _int, _i64, _i64, _int, _vp, _vp, _i64, _vp, _vp, _vp]),
     "rpbh_packed_bytes": (_i64, [_i64, _i64, _int]),
     "wq_gaussian_lloyd_max": (_int, [_int, _int, _vp]),
     "wq_rpbh_codebook": (_int, [_int, _i64, _vp]),
@@ -193,6 +194,21 @@ def rpbh_rotate_activations(x: torch.Tensor, perm: torch.Tensor, signs: torch.Te
     st = lib().rpbh_rotate_activations(_dev(x, "x"), _DT.get(x.dtype, -1), rows, d, _dev(perm, "perm"),
                                        _dev(signs, "signs"), _dev(out, "out"), _stream(x.device))
     _check("rpbh_rotate_activations", st)
+    return out
+
+
+def rpbh_linear(packed: torch.Tensor, row_norms: torch.Tensor, out_features: int, d: int, bits: int, codebook,
+                x_rot: torch.Tensor, bias=None, out=None):
+    """y = x_rot W'^T + bias [m, out_features] bf16, W' the rotated dequantized weight of `packed`."""
+    cb = _codebook_arg(codebook, bits)
+    m = x_rot.shape[0]
+    if out is None:
+        out = torch.empty(m, out_features, dtype=torch.bfloat16, device=x_rot.device)
+    bp = _dev(bias, "bias") if bias is not None else None
+    st = lib().rpbh_linear(_dev(packed, "packed"), _dev(row_norms, "row_norms"), _DT.get(row_norms.dtype, -1),
+                           out_features, d, bits, cb.ctypes.data, _dev(x_rot, "x_rot"), m, bp, _dev(out, "y"),
+                           _stream(x_rot.device))
+    _check("rpbh_linear", st)
     return out
 
 
