@@ -3,13 +3,15 @@
 // (_dequantize_rotated: codebook[codes] * norms in the weight dtype). W' is never written out: its
 // packed codes are unpacked straight into the tensor-core operand in shared memory.
 //
-// One CTA computes a 128 x 256 tile of D = W'_tile x_rot_tile^T (128 output features = the
-// product's M and the accumulator's lanes, 256 activation rows = N and its columns), K = d in
-// chunks of 64 (one 128-byte swizzle atom of bf16):
+// One CTA computes a 256 x 256 tile of D = W'_tile x_rot_tile^T (256 output features as two
+// halves of 128 = the product's M and the accumulators' lanes, 256 activation rows = N and their
+// columns), K = d in chunks of 64 (one 128-byte swizzle atom of bf16); the two halves share each
+// x_rot tile, so x_rot is read once per 256 output features:
 //   * warp 0, lane 0: TMA loads of x_rot [256 x 64] bf16 tiles (128-byte swizzle) into a ring of
-//     four stages, and the products: four tcgen05.mma.kind::f16 (M = 128, N = 256, K = 16) per
-//     chunk, accumulating in 256 tensor-memory columns, each chunk's commit releasing its stage;
-//   * warps 4..7: thread p owns output feature n0 + p: it loads the chunk's 8 * bits code bytes
+//     three stages, and the products: per chunk and K = 16 step one tcgen05.mma.kind::f16
+//     (M = 128, N = 256) per half, accumulating in 2 x 256 tensor-memory columns, each chunk's
+//     commit releasing its stage;
+//   * warps 4..11: thread p owns output feature n0 + p: it loads the chunk's 8 * bits code bytes
 //     of its row, unpacks the 64 codes (MSB-first stream, pack_codes) and looks each up in the
 //     codebook rounded to bf16 (a shuffle: lane l holds centroid l mod 2^bits), writing the 128-byte
 //     row of the operand tile with the 128-byte swizzle; then, after the last product, the
@@ -35,21 +37,24 @@
 namespace wq {
 namespace rpbh_linear {
 
-constexpr int kTM = 128;  // output features per tile
+constexpr int kTM = 256;  // output features per tile (two halves of 128: the product's M)
 constexpr int kTN = 256;  // activation rows per tile
 constexpr int kTK = 64;   // K per chunk
-constexpr int kStages = 4;
-constexpr int kThreads = 256;
+constexpr int kStages = 3;
+constexpr int kProducerWarps = kTM / 32;
+constexpr int kThreads = 128 + 32 * kProducerWarps;
+constexpr int kAHalf = 128 * kTK * 2;  // one half of the weight tile
 constexpr int kABytes = kTM * kTK * 2;
 constexpr int kBBytes = kTN * kTK * 2;
 constexpr int kOffA = 0;
 constexpr int kOffB = kStages * kABytes;
-constexpr int kOffBar = kOffB + kStages * kBBytes;  // full_a[4], full_b[4], empty[4], done, then the TMEM address
+constexpr int kOffBar = kOffB + kStages * kBBytes;  // full_a, full_b, empty (per stage), done, then the TMEM address
 constexpr int kSmem = 1024 + kOffBar + 8 * (3 * kStages + 1) + 16;
 static_assert(kSmem <= 232448, "the ring must fit the 227 KB a CTA may use");
 // fp32 accumulator, bf16 A and B, both K-major, N = 256, M = 128
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTN >> 3) << 17) |
-                            ((uint32_t)(kTM >> 4) << 24);
+                            ((uint32_t)(128 >> 4) << 24);
+constexpr uint32_t kTmemCols = 2 * kTN;
 constexpr uint32_t kMaxPolls = 1u << 24;
 
 __device__ unsigned int g_fault;
@@ -82,20 +87,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kTM, m0 = blockIdx.y * kTN;
     const int nchunks = d / kTK;
-    uint64_t *const full_a = reinterpret_cast<uint64_t *>(base + kOffBar);  // the 4 unpacking warps arrive
+    uint64_t *const full_a = reinterpret_cast<uint64_t *>(base + kOffBar);  // the unpacking warps arrive
     uint64_t *const full_b = full_a + kStages;                             // the TMA of x_rot lands
     uint64_t *const empty = full_b + kStages;                              // the chunk's products are done
     uint64_t *const done = empty + kStages;                                // every product is done
     uint32_t *const tslot = reinterpret_cast<uint32_t *>(done + 1);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full_a[s], 4);
+            mbar_init(&full_a[s], kProducerWarps);
             mbar_init(&full_b[s], 1);
             mbar_init(&empty[s], 1);
         }
         mbar_init(done, 1);
     }
-    if (warp == 0) tmem_alloc(tslot, kTN);
+    if (warp == 0) tmem_alloc(tslot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -104,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            uint32_t issued[kStages] = {0u, 0u, 0u, 0u};  // x_rot copies issued per stage (fault path)
+            uint32_t issued[kStages] = {};  // x_rot copies issued per stage (fault path)
             auto load_b = [&](int c) {
                 const int s = c % kStages;
                 mbar_expect_tx(&full_b[s], kBBytes);
@@ -123,8 +128,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t ad = sw128_desc(smem_u32(base + kOffA + s * kABytes));
                 const uint64_t bd = sw128_desc(smem_u32(base + kOffB + s * kBBytes));
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // K = 16 per instruction: 32 bytes into each 128-byte row
-                    mma_bf16(tmem, ad + (uint32_t)(ks * 2), bd + (uint32_t)(ks * 2), kIdesc, (c > 0 || ks > 0) ? 1u : 0u);
+                for (int ks = 0; ks < 4; ++ks) {  // K = 16 per instruction: 32 bytes into each 128-byte row
+                    const uint32_t acc = (c > 0 || ks > 0) ? 1u : 0u;
+                    mma_bf16(tmem, ad + (uint32_t)(ks * 2), bd + (uint32_t)(ks * 2), kIdesc, acc);
+                    mma_bf16(tmem + (uint32_t)kTN, ad + (uint32_t)((kAHalf >> 4) + ks * 2), bd + (uint32_t)(ks * 2),
+                             kIdesc, acc);
+                }
                 mma_commit(&empty[s]);
                 // the previous chunk's stage takes the chunk kStages after it once its products are done
                 if (c >= 1 && c - 1 + kStages < nchunks) {
@@ -151,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint8_t *const src = packed + (int64_t)(valid ? n : 0) * (d / 8 * BITS);
         // lane l holds the bf16 centroid l mod 2^bits: a shuffle from the lane named by a code is the lookup
         const uint32_t cbv = cb.c[lane & ((1 << BITS) - 1)];
-        unsigned char *const rowA = base + kOffA + p * 128;
+        unsigned char *const rowA = base + kOffA + (p >> 7) * kAHalf + (p & 127) * 128;
         const int sw = p & 7;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
@@ -196,7 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             rho = bf16_to_f32(f32_to_bf16(rho));
             if (bias) b = bf16_to_f32(bias[n]);
         }
-        const uint32_t lanes = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        // warps 4..7 read the first half's accumulator, warps 8..11 the second's (lanes 32 (warp % 4) ..)
+        const uint32_t lanes = tmem + (uint32_t)((p >> 7) * kTN) + ((uint32_t)((warp & 3) * 32) << 16);
 #pragma unroll 1
         for (int j = 0; j < kTN / 32; ++j) {
             float v[32];
@@ -214,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTN);
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
