@@ -162,6 +162,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t cbv = cb.c[lane & ((1 << BITS) - 1)];
         unsigned char *const rowA = base + kOffA + (p >> 7) * kAHalf + (p & 127) * 128;
         const int sw = p & 7;
+        // the code bytes of chunk c + 2 are loaded while chunk c is unpacked (two register sets
+        // ahead, so the loads' latency is hidden behind two chunks of work)
+        uint2 raw[2][BITS];
+        auto fetch = [&](int c, uint2 (&r)[BITS]) {
+#pragma unroll
+            for (int q = 0; q < BITS; ++q)
+                r[q] = c < nchunks ? __ldg(reinterpret_cast<const uint2 *>(src + c * 8 * BITS) + q) : make_uint2(0u, 0u);
+        };
+        fetch(0, raw[0]);
+        fetch(1, raw[1]);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % kStages;
             if (c >= kStages && !fault) {
@@ -173,10 +183,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t W[2 * BITS];
 #pragma unroll
             for (int q = 0; q < BITS; ++q) {
-                const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src + c * 8 * BITS) + q);
+                const uint2 v = (c & 1) ? raw[1][q] : raw[0][q];
                 W[2 * q] = __byte_perm(v.x, 0u, 0x0123);
                 W[2 * q + 1] = __byte_perm(v.y, 0u, 0x0123);
             }
+            if (c & 1)
+                fetch(c + 2, raw[1]);
+            else
+                fetch(c + 2, raw[0]);
             unsigned char *const A = rowA + s * kABytes;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {  // 16-byte chunk j: k = 8j .. 8j + 7
