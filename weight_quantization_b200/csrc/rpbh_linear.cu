@@ -38,24 +38,31 @@ namespace wq {
 namespace rpbh_linear {
 
 constexpr int kTM = 256;  // output features per tile (two halves of 128: the product's M)
-constexpr int kTN = 256;  // activation rows per tile
 constexpr int kTK = 64;   // K per chunk
 constexpr int kStages = 3;
 constexpr int kProducerWarps = kTM / 32;
 constexpr int kThreads = 128 + 32 * kProducerWarps;
 constexpr int kAHalf = 128 * kTK * 2;  // one half of the weight tile
 constexpr int kABytes = kTM * kTK * 2;
-constexpr int kBBytes = kTN * kTK * 2;
 constexpr int kOffA = 0;
 constexpr int kOffB = kStages * kABytes;
-constexpr int kOffBar = kOffB + kStages * kBBytes;  // full_a, full_b, empty (per stage), done, then the TMEM address
-constexpr int kSmem = 1024 + kOffBar + 8 * (3 * kStages + 1) + 16;
-static_assert(kSmem <= 232448, "the ring must fit the 227 KB a CTA may use");
-// fp32 accumulator, bf16 A and B, both K-major, N = 256, M = 128
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTN >> 3) << 17) |
-                            ((uint32_t)(128 >> 4) << 24);
-constexpr uint32_t kTmemCols = 2 * kTN;
+constexpr uint32_t kTmemCols = 512;  // the two accumulators at columns 0 and 256
 constexpr uint32_t kMaxPolls = 1u << 24;
+
+// TN activation rows per tile (the product's N: a multiple of 16 up to 256; the host picks the
+// one that fills the SMs best)
+template <int TN>
+struct Tile {
+    static constexpr int kTN = TN;
+    static constexpr int kBBytes = TN * kTK * 2;
+    static constexpr int kOffBar = kOffB + kStages * kBBytes;  // full_a, full_b, empty (per stage), done, TMEM address
+    static constexpr int kSmem = 1024 + kOffBar + 8 * (3 * kStages + 1) + 16;
+    static_assert(TN % 16 == 0 && TN <= 256 && kBBytes % 1024 == 0, "N of one tcgen05.mma, whole swizzle atoms");
+    static_assert(kSmem <= 232448, "the ring must fit the 227 KB a CTA may use");
+    // fp32 accumulator, bf16 A and B, both K-major, N = TN, M = 128
+    static constexpr uint32_t kIdesc =
+        (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(TN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+};
 
 __device__ unsigned int g_fault;
 
@@ -77,11 +84,14 @@ __device__ __forceinline__ uint32_t code_at(const uint32_t (&W)[2 * BITS], int i
     return __funnelshift_l(W[q + 1], W[q], r + BITS - 32) & kMask;
 }
 
-template <int BITS, bool kNormBf16>
+template <int BITS, bool kNormBf16, int TN>
 __global__ void __launch_bounds__(kThreads, 1)
     linear_kernel(const uint8_t *__restrict__ packed, const void *__restrict__ row_norms, int out_f, int d,
                   const __grid_constant__ CUtensorMap xmap, int m_rows, const uint16_t *__restrict__ bias,
                   CodebookBf16 cb, uint16_t *__restrict__ y) {
+    using T = Tile<TN>;
+    constexpr int kTN = TN, kBBytes = T::kBBytes, kOffBar = T::kOffBar;
+    constexpr uint32_t kIdesc = T::kIdesc;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *const base = align1024(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -131,8 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int ks = 0; ks < 4; ++ks) {  // K = 16 per instruction: 32 bytes into each 128-byte row
                     const uint32_t acc = (c > 0 || ks > 0) ? 1u : 0u;
                     mma_bf16(tmem, ad + (uint32_t)(ks * 2), bd + (uint32_t)(ks * 2), kIdesc, acc);
-                    mma_bf16(tmem + (uint32_t)kTN, ad + (uint32_t)((kAHalf >> 4) + ks * 2), bd + (uint32_t)(ks * 2),
-                             kIdesc, acc);
+                    mma_bf16(tmem + 256u, ad + (uint32_t)((kAHalf >> 4) + ks * 2), bd + (uint32_t)(ks * 2), kIdesc,
+                             acc);
                 }
                 mma_commit(&empty[s]);
                 // the previous chunk's stage takes the chunk kStages after it once its products are done
@@ -220,16 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (bias) b = bf16_to_f32(bias[n]);
         }
         // warps 4..7 read the first half's accumulator, warps 8..11 the second's (lanes 32 (warp % 4) ..)
-        const uint32_t lanes = tmem + (uint32_t)((p >> 7) * kTN) + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t lanes = tmem + (uint32_t)((p >> 7) * 256) + ((uint32_t)((warp & 3) * 32) << 16);
 #pragma unroll 1
-        for (int j = 0; j < kTN / 32; ++j) {
+        for (int j = 0; j < (kTN + 31) / 32; ++j) {
             float v[32];
-            tmem_ld32(lanes + 32u * j, v);
+            tmem_ld32(lanes + 32u * j, v);  // (past column kTN the values are not this tile's: not stored)
             tmem_wait(v);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const int m = m0 + 32 * j + i;
-                if (valid && m < m_rows) y[(int64_t)m * out_f + n] = f32_to_bf16(__fmaf_rn(v[i], rho, b));
+                if (valid && 32 * j + i < kTN && m < m_rows) y[(int64_t)m * out_f + n] = f32_to_bf16(__fmaf_rn(v[i], rho, b));
             }
         }
     }
@@ -254,19 +264,41 @@ uint16_t bf16_rne(float f) {
     return (uint16_t)(u >> 16);
 }
 
-template <int BITS, bool kNB>
-wq_status launch(const uint8_t *packed, const void *row_norms, int64_t out_f, int64_t d, const CUtensorMap &xm,
-                 int64_t m, const uint16_t *bias, const CodebookBf16 &cb, uint16_t *y, cudaStream_t s) {
-    auto k = linear_kernel<BITS, kNB>;
-    if (!ensure_dynamic_smem(reinterpret_cast<const void *>(k), kSmem)) return WQ_ERR_CUDA;
-    const dim3 grid((unsigned)((out_f + kTM - 1) / kTM), (unsigned)((m + kTN - 1) / kTN));
-    k<<<grid, kThreads, kSmem, s>>>(packed, row_norms, (int)out_f, (int)d, xm, (int)m, bias, cb, y);
+template <int BITS, bool kNB, int TN>
+wq_status launch_tn(const uint8_t *packed, const void *row_norms, int64_t out_f, int64_t d, const void *x_rot,
+                    int64_t m, const uint16_t *bias, const CodebookBf16 &cb, uint16_t *y, cudaStream_t s) {
+    CUtensorMap xm;
+    if (!make_tmap_2d(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_rot, (uint64_t)d, (uint64_t)m, (uint64_t)d * 2, kTK, TN))
+        return WQ_ERR_CUDA;
+    auto k = linear_kernel<BITS, kNB, TN>;
+    if (!ensure_dynamic_smem(reinterpret_cast<const void *>(k), Tile<TN>::kSmem)) return WQ_ERR_CUDA;
+    const dim3 grid((unsigned)((out_f + kTM - 1) / kTM), (unsigned)((m + TN - 1) / TN));
+    k<<<grid, kThreads, Tile<TN>::kSmem, s>>>(packed, row_norms, (int)out_f, (int)d, xm, (int)m, bias, cb, y);
     return launch_status();
+}
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (!cached[dev]) cudaDeviceGetAttribute(&cached[dev], cudaDevAttrMultiProcessorCount, dev);
+    return cached[dev];
+}
+
+// One CTA per SM: a tile width of 240 rows instead of 256 is taken when it needs fewer rounds of
+// CTAs times the width (e.g. 16 x 9 = 144 tiles in one round on 148 SMs instead of 16 x 8 = 128).
+template <int BITS, bool kNB>
+wq_status launch(const uint8_t *packed, const void *row_norms, int64_t out_f, int64_t d, const void *x_rot,
+                 int64_t m, const uint16_t *bias, const CodebookBf16 &cb, uint16_t *y, cudaStream_t s) {
+    const int64_t sms = sm_count() > 0 ? sm_count() : 1, tn = (out_f + kTM - 1) / kTM;
+    auto cost = [&](int64_t w) { return ((tn * ((m + w - 1) / w) + sms - 1) / sms) * w; };
+    if (cost(240) < cost(256)) return launch_tn<BITS, kNB, 240>(packed, row_norms, out_f, d, x_rot, m, bias, cb, y, s);
+    return launch_tn<BITS, kNB, 256>(packed, row_norms, out_f, d, x_rot, m, bias, cb, y, s);
 }
 
 template <bool kNB>
 wq_status by_bits(int bits, const uint8_t *packed, const void *row_norms, int64_t out_f, int64_t d,
-                  const CUtensorMap &xm, int64_t m, const uint16_t *bias, const CodebookBf16 &cb, uint16_t *y,
+                  const void *xm, int64_t m, const uint16_t *bias, const CodebookBf16 &cb, uint16_t *y,
                   cudaStream_t s) {
     switch (bits) {
         case 2: return launch<2, kNB>(packed, row_norms, out_f, d, xm, m, bias, cb, y, s);
@@ -305,10 +337,7 @@ extern "C" wq_status rpbh_linear(const uint8_t *packed, const void *row_norms, i
         return WQ_ERR_ALIGN;
     rpbh_linear::CodebookBf16 cb = {};
     for (int k = 0; k < (1 << bits); ++k) cb.c[k] = rpbh_linear::bf16_rne(codebook[k]);
-    CUtensorMap xm;
-    if (!make_tmap_2d(&xm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x_rot, (uint64_t)d, (uint64_t)m, (uint64_t)d * 2,
-                      rpbh_linear::kTK, rpbh_linear::kTN))
-        return WQ_ERR_CUDA;
+    const void *xm = x_rot;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const auto *b = static_cast<const uint16_t *>(bias);
     auto *yo = static_cast<uint16_t *>(y);
