@@ -75,13 +75,14 @@ __device__ __forceinline__ unsigned char *align1024(unsigned char *p) {
 }
 
 // Code i (0 .. 63) of a chunk whose 8 * BITS bytes are held as big-endian 32-bit words W
-// (stream bit b is bit 31 - b % 32 of W[b / 32]).
+// (stream bit b is bit 31 - b % 32 of W[b / 32]), in the low BITS bits of the result; the bits
+// above it are whatever follows in the word. A shuffle takes its source lane modulo 32, and lane l
+// holds centroid l mod 2^BITS, so the lookup needs no mask.
 template <int BITS>
 __device__ __forceinline__ uint32_t code_at(const uint32_t (&W)[2 * BITS], int i) {
     const int o = BITS * i, q = o >> 5, r = o & 31;
-    constexpr uint32_t kMask = (1u << BITS) - 1u;
-    if (r + BITS <= 32) return (W[q] >> (32 - r - BITS)) & kMask;
-    return __funnelshift_l(W[q + 1], W[q], r + BITS - 32) & kMask;
+    if (r + BITS <= 32) return W[q] >> (32 - r - BITS);
+    return __funnelshift_l(W[q + 1], W[q], r + BITS - 32);
 }
 
 template <int BITS, bool kNormBf16, int TN>
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int u = 0; u < 4; ++u) {
                     const uint32_t lo = __shfl_sync(0xffffffffu, cbv, (int)code_at<BITS>(W, 8 * j + 2 * u));
                     const uint32_t hi = __shfl_sync(0xffffffffu, cbv, (int)code_at<BITS>(W, 8 * j + 2 * u + 1));
-                    w4[u] = valid ? (lo | (hi << 16)) : 0u;
+                    w4[u] = __byte_perm(lo, hi, 0x5410);  // (rows past out_features: never stored)
                 }
                 *reinterpret_cast<uint4 *>(A + ((j ^ sw) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
