@@ -198,10 +198,18 @@ wq_status wq_rpbh_codebook(int bits, int64_t d, float *out);
  * bounded wait runs out (which does not happen in normal operation) sets a bit and returns early,
  * leaving its outputs unspecified: bit 0 a TQ3 kernel waiting for a TMA tile, bit 1 an RPBH kernel
  * waiting for a row copy, bit 3 the tensor-core TQ3 encoder waiting for a tile or its product,
- * bit 4 rpbh_linear waiting for a tile, the unpacked weights or its product.
+ * bit 4 rpbh_linear waiting for a tile, the unpacked weights or its product, bit 5 the self-test
+ * wq_selftest_wait_timeout.
  * Synchronous (a device-to-host copy on the legacy default stream); `flags` is host memory.
  * Errors: WQ_ERR_NULL, WQ_ERR_CUDA. */
 wq_status wq_device_fault(unsigned int *flags);
+
+/* wq_selftest_wait_timeout -- exercises the fault path without a GPU fault (no counterpart in the
+ * pages): one thread waits, with the library's bounded wait, on an mbarrier that nothing arrives
+ * at; after the wait's 2 s limit it sets fault bit 5 and returns, so wq_device_fault then reports
+ * 32 and the context stays usable. Enqueued on `stream`; takes about 2 s of GPU time.
+ * Errors: WQ_ERR_CUDA. */
+wq_status wq_selftest_wait_timeout(void *stream);
 
 /* wq_status_string -- a static, NUL-terminated description of a status code. */
 const char *wq_status_string(int status);

@@ -479,6 +479,23 @@ extern "C" int64_t tq3_compressed_bytes(int64_t n_vec) {
     return n_vec * 56;
 }
 
+namespace wq {
+namespace tq3 {
+// One thread waits, through the same bounded wait the kernels use, on an mbarrier that nothing
+// arrives at; when the wait gives up (after 2 s of %globaltimer) it sets fault bit 5 and returns.
+__global__ void selftest_wait_kernel() {
+    __shared__ uint64_t bar;
+    mbar_init(&bar, 1);
+    if (!mbar_wait_bounded(&bar, 0u, 1u << 30)) atomicOr(&g_fault, 32u);
+}
+}  // namespace tq3
+}  // namespace wq
+
+extern "C" wq_status wq_selftest_wait_timeout(void *stream) {
+    wq::tq3::selftest_wait_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>();
+    return launch_status();
+}
+
 extern "C" wq_status wq_device_fault(unsigned int *flags) {
     if (!flags) return WQ_ERR_NULL;
     unsigned int v = 0, zero = 0;

@@ -34,6 +34,7 @@ PROTOTYPES = {
     "wq_gaussian_lloyd_max": (_int, [_int, _int, _vp]),
     "wq_rpbh_codebook": (_int, [_int, _i64, _vp]),
     "wq_device_fault": (_int, [_vp]),
+    "wq_selftest_wait_timeout": (_int, [_vp]),
     "wq_status_string": (C.c_char_p, [_int]),
     "wq_version": (_int, []),
 }
@@ -219,6 +220,11 @@ def gaussian_lloyd_max(bits: int, iters: int = 200) -> np.ndarray:
     out = np.zeros(1 << bits, np.float32)
     _check("wq_gaussian_lloyd_max", lib().wq_gaussian_lloyd_max(bits, iters, out.ctypes.data))
     return out
+
+
+def selftest_wait_timeout(device=None):
+    """Runs the library's bounded-wait self-test on the current stream (about 2 s of GPU time)."""
+    _check("wq_selftest_wait_timeout", lib().wq_selftest_wait_timeout(_stream(device or torch.cuda.current_device())))
 
 
 def device_fault() -> int:
