@@ -96,6 +96,17 @@ wq_status tq3_encode_exact(const void *x, int x_dtype, int64_t n_vec, const uint
 wq_status tq3_decode(const uint8_t *packed, const float *norms, const float *scales, int64_t n_vec,
                      const uint32_t *sign_mask, void *out, int out_dtype, void *stream);
 
+/* tq3_encode_aos / tq3_decode_aos -- tq3_encode and tq3_decode on 56-byte records (the "56 bytes
+ * per vector" of tq3_memory_bytes as one array of structures): record v is the 48 packed bytes,
+ * then the norm, then the scale (fp32, little-endian), at byte 56 v. Same arithmetic, precision and
+ * errors as the three-array forms.
+ *   records    device, n_vec x 56 bytes, 8-byte aligned.
+ *   x, out     device, n_vec x 128 elements, 16-byte aligned. */
+wq_status tq3_encode_aos(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
+                         uint8_t *records, void *stream);
+wq_status tq3_decode_aos(const uint8_t *records, int64_t n_vec, const uint32_t *sign_mask, void *out,
+                         int out_dtype, void *stream);
+
 /* tq3_compressed_bytes -- tq3_memory_bytes' compressed size for n_vec vectors: 56 * n_vec
  * (-1 if n_vec < 0 or the product overflows). */
 int64_t tq3_compressed_bytes(int64_t n_vec);

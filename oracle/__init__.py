@@ -140,6 +140,22 @@ def tq3_unpack(packed):
     return out
 
 
+def tq3_to_records(packed, norms, scales):
+    """The 56-byte record of each vector ("56 bytes per vector", tq3_memory_bytes): its 48 packed bytes,
+    then the fp32 norm and the fp32 scale, little-endian."""
+    p = np.ascontiguousarray(packed, np.uint8).reshape(-1, 48)
+    n = np.ascontiguousarray(norms, '<f4').reshape(-1, 1).view(np.uint8)
+    s = np.ascontiguousarray(scales, '<f4').reshape(-1, 1).view(np.uint8)
+    return np.concatenate([p, n, s], axis=1)
+
+
+def tq3_from_records(records):
+    """The inverse of tq3_to_records: (packed [n, 48], norms [n], scales [n])."""
+    r = np.ascontiguousarray(records, np.uint8).reshape(-1, 56)
+    return (r[:, :48].copy(), r[:, 48:52].copy().view('<f4').reshape(-1).astype(np.float32),
+            r[:, 52:56].copy().view('<f4').reshape(-1).astype(np.float32))
+
+
 def tq3_memory_bytes(shape):
     s = np.asarray(shape, dtype=np.int64)
     orig = np.zeros(1, np.int64)

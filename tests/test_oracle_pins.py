@@ -468,6 +468,22 @@ def test_rpbh_dequantize_matches_dense(oracle):
     assert np.abs(w - wrot.astype(np.float64) @ R).max() < 1e-5
 
 
+def test_tq3_records_are_the_pages_56_bytes(oracle):
+    """A record is the page's compressed size per vector (tq3_memory_bytes: 56 bytes), laid out as
+    the 48 packed bytes, then the norm and the scale as little-endian fp32; the split is exact."""
+    import struct
+    comp, _, _ = oracle.tq3_memory_bytes((3, 128))
+    x = inputs.gaussian((3, 128), seed=75).astype(np.float32)
+    p, n, sc = oracle.tq3_encode(x, inputs.tq3_sign_bits())
+    r = oracle.tq3_to_records(p, n, sc)
+    assert r.shape == (3, 56) and r.size == comp
+    for v in range(3):
+        assert bytes(r[v, :48]) == bytes(p[v])
+        assert bytes(r[v, 48:]) == struct.pack('<ff', float(n[v]), float(sc[v]))
+    p2, n2, s2 = oracle.tq3_from_records(r)
+    assert np.array_equal(p2, p) and np.array_equal(n2, n) and np.array_equal(s2, sc)
+
+
 def test_rpbh_linear_one_hot_and_zero_inputs(oracle):
     """forward's F.linear on the rotated activations: a one-hot activation row e_k returns column k
     of the bf16 rotated weight plus the bias (so the product is x W'^T, not a transpose of it), and

@@ -1,12 +1,13 @@
-// TQ3 KV-cache codec on sm_100a: page "tq3_core.py" (tq3_quantize, tq3_dequantize).
+// TQ3 KV-cache codec on sm_100a: page "tq3_core.py" (tq3_quantize, tq3_dequantize). This file
+// holds the C ABI of the TQ3 entry points and the step-by-step encoder behind tq3_encode_exact;
+// the fast encoders are in tq3_mma.cu (bf16) and tq3_rows.cu (fp32), the decoder in tq3_rows.cu.
 //
-// Layout: two threads own one 128-element vector. Lanes 0-15 of a warp hold elements 0..63 of 16
-// vectors and lanes 16-31 hold elements 64..127 of the same vectors, so six of the seven FWHT
-// stages run in registers and only the last one (h = 64) exchanges values with a shuffle. A CTA of
-// 128 threads handles 64 vectors. The encoder's input tile is loaded from HBM by TMA into shared
-// memory with 128-byte swizzling; the decoder stages its output tile in the same swizzled layout
-// and writes it back with coalesced 16-byte stores. Either way every thread reads or writes its
-// own 128-byte row segment without bank conflicts and global traffic is whole, contiguous tiles.
+// Step-by-step encoder layout: two threads own one 128-element vector. Lanes 0-15 of a warp hold
+// elements 0..63 of 16 vectors and lanes 16-31 hold elements 64..127 of the same vectors, so six of
+// the seven FWHT stages run in registers and only the last one (h = 64) exchanges values with a
+// shuffle. A CTA of 128 threads handles 64 vectors; its input tile is loaded from HBM by TMA into
+// shared memory with 128-byte swizzling, so every thread reads its own 128-byte row segment
+// without bank conflicts and global traffic is whole, contiguous tiles.
 //
 // Rounding follows the page step by step in fp32 (the library is built with -fmad=false; fused
 // operations are written explicitly only where they are exact), so packed bytes, norms and scales
@@ -267,118 +268,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     }
 }
 
-template <bool kBf16Out, bool kDefault>
-__global__ void __launch_bounds__(kThreads, 4)
-    decode_kernel(const uint8_t *__restrict__ packed, const float *__restrict__ norms,
-                  const float *__restrict__ scales, int64_t n_vec, SignMask mask, void *__restrict__ out) {
-    constexpr int kBoxes = kBf16Out ? 2 : 4;
-    extern __shared__ unsigned char smem_raw[];
-    __shared__ float ctab[8];
-    unsigned char *tile = tile_base(smem_raw);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int half = lane >> 4;
-    const int row = warp * 16 + (lane & 15);
-    const int64_t v = (int64_t)blockIdx.x * kRows + row;
-    if (threadIdx.x < 8) ctab[threadIdx.x] = centroid(threadIdx.x);
-
-    // this thread's 64 indices: bytes 24 * half .. 24 * half + 23 of the 48-byte record
-    uint32_t pw[6] = {0, 0, 0, 0, 0, 0};
-    float n = 0.0f, scale = 0.0f;
-    if (v < n_vec) {
-        // bytes 48v + 24 * half ... as one 16-byte chunk at 48v + 32 * half and one 8-byte chunk at
-        // 48v + 16 + 8 * half: aligned for either half, no lane-divergent branch around the loads
-        const uint8_t *rec = packed + v * 48;
-        const uint4 c16 = ld_stream16(rec + 32 * half);
-        const uint2 c8 = ld_stream8(rec + 16 + 8 * half);
-        pw[0] = half ? c8.x : c16.x;
-        pw[1] = half ? c8.y : c16.y;
-        pw[2] = half ? c16.x : c16.z;
-        pw[3] = half ? c16.y : c16.w;
-        pw[4] = half ? c16.z : c8.x;
-        pw[5] = half ? c16.w : c8.y;
-        n = norms[v];
-        scale = scales[v];
-    }
-    __syncthreads();  // ctab
-
-    // _unpack_3bit, then centroids[idx] * scale
-    float a[64];
-#pragma unroll
-    for (int c2 = 0; c2 < 2; ++c2) {
-        const uint32_t w0 = pw[3 * c2], w1 = pw[3 * c2 + 1], w2 = pw[3 * c2 + 2];
-        const uint32_t g[4] = {w0 & 0xffffffu, (w0 >> 24) | ((w1 & 0xffffu) << 8), (w1 >> 16) | ((w2 & 0xffu) << 16),
-                               w2 >> 8};
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) a[32 * c2 + 8 * k + i] = __fmul_rn(ctab[(g[k] >> (3 * i)) & 7u], scale);
-    }
-    // the normalised FWHT (its own inverse)
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-        const float p = a[2 * k], q = a[2 * k + 1];
-        a[2 * k] = __fadd_rn(p, q);
-        a[2 * k + 1] = __fsub_rn(p, q);
-    }
-    fwht_local_2_32(a);
-#pragma unroll
-    for (int i = 0; i < 64; ++i) {
-        const float o = __shfl_xor_sync(0xffffffffu, a[i], 16);
-        a[i] = half ? __fsub_rn(o, a[i]) : __fadd_rn(a[i], o);
-    }
-    // * post, then * norm; the sign flips (exact) are applied to the output bits
-    {
-        const float post = fwht_post();
-        const f32x2 P2 = pk2(post, post), N2 = pk2(n, n);
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-            upk2(mul2(mul2(pk2(a[2 * k], a[2 * k + 1]), P2), N2), a[2 * k], a[2 * k + 1]);
-    }
-    const uint32_t H = half ? 0xffffffffu : 0u;
-    const uint32_t mlo = half ? mask.w[2] : mask.w[0], mhi = half ? mask.w[3] : mask.w[1];
-    if (kBf16Out) {
-        unsigned char *box = tile + half * kBoxBytes;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            uint32_t o[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int k = 4 * j + u;
-                o[u] = pack_bf16x2(a[2 * k], a[2 * k + 1]) ^ pair_flip<kDefault>(k, H, mlo, mhi);
-            }
-            *reinterpret_cast<uint4 *>(swz(box, row, j)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            unsigned char *box = tile + (2 * half + (j >> 3)) * kBoxBytes;
-            uint32_t o[4];
-#pragma unroll
-            for (int u = 0; u < 4; u += 2) {
-                const int k = 2 * j + u / 2;
-                const uint32_t f = pair_flip<kDefault>(k, H, mlo, mhi);
-                o[u] = __float_as_uint(a[2 * k]) ^ (f << 16);
-                o[u + 1] = __float_as_uint(a[2 * k + 1]) ^ (f & 0x80000000u);
-            }
-            *reinterpret_cast<uint4 *>(swz(box, row, j & 7)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-    }
-    __syncthreads();
-    // write the tile back with coalesced 16-byte stores: the CTA's rows are one contiguous range
-    constexpr int kChunksPerRow = kBoxes * 8;
-    const int64_t rows_left = n_vec - (int64_t)blockIdx.x * kRows;
-    unsigned char *gdst = static_cast<unsigned char *>(out) + (int64_t)blockIdx.x * kRows * (kChunksPerRow * 16);
-#pragma unroll
-    for (int it = 0; it < kChunksPerRow * kRows / kThreads; ++it) {
-        const int chunk = it * kThreads + threadIdx.x;
-        const int r = chunk / kChunksPerRow, cj = chunk % kChunksPerRow;
-        if (r < rows_left) {
-            const uint4 val = *reinterpret_cast<const uint4 *>(swz(tile + (cj >> 3) * kBoxBytes, r, cj & 7));
-            st_stream16(gdst + (int64_t)chunk * 16, val);
-        }
-    }
-}
-
+// Dynamic shared memory of the step-by-step encoder: the input tile plus alignment and barrier.
 inline size_t smem_bytes(bool bf16) { return (size_t)(bf16 ? 2 : 4) * kBoxBytes + 1024 + 64; }
 
 }  // namespace tq3
@@ -450,28 +340,35 @@ extern "C" wq_status tq3_decode(const uint8_t *packed, const float *norms, const
     tq3::SignMask m;
     for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
     return tq3_rows::decode(packed, norms, scales, n_vec, m, out, out_dtype, static_cast<cudaStream_t>(stream));
-    const bool def = tq3::is_default(m), bf = out_dtype == WQ_BF16;
-    const int esz = bf ? 2 : 4;
-    const size_t smem = tq3::smem_bytes(bf);
+}
+
+extern "C" wq_status tq3_encode_aos(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
+                                    uint8_t *records, void *stream) {
+    if (n_vec < 0) return WQ_ERR_SHAPE;
+    if (!valid_dtype(x_dtype)) return WQ_ERR_DTYPE;
+    if (n_vec == 0) return WQ_OK;
+    if (!x || !sign_mask || !records) return WQ_ERR_NULL;
+    if (n_vec > ((int64_t)1 << 40)) return WQ_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(records, 8)) return WQ_ERR_ALIGN;
+    tq3::SignMask m;
+    for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    for (int64_t off = 0; off < n_vec; off += tq3::kMaxChunk) {
-        const int64_t cnt = n_vec - off < tq3::kMaxChunk ? n_vec - off : tq3::kMaxChunk;
-        unsigned char *oc = static_cast<unsigned char *>(out) + off * (tq3::kD * esz);
-        const unsigned grid = (unsigned)((cnt + tq3::kRows - 1) / tq3::kRows);
-        const uint8_t *pc = packed + off * 48;
-        const float *nc = norms + off, *sc = scales + off;
-        if (bf && def)
-            tq3::decode_kernel<true, true><<<grid, tq3::kThreads, smem, s>>>(pc, nc, sc, cnt, m, oc);
-        else if (bf)
-            tq3::decode_kernel<true, false><<<grid, tq3::kThreads, smem, s>>>(pc, nc, sc, cnt, m, oc);
-        else if (def)
-            tq3::decode_kernel<false, true><<<grid, tq3::kThreads, smem, s>>>(pc, nc, sc, cnt, m, oc);
-        else
-            tq3::decode_kernel<false, false><<<grid, tq3::kThreads, smem, s>>>(pc, nc, sc, cnt, m, oc);
-        const wq_status st = launch_status();
-        if (st != WQ_OK) return st;
-    }
-    return WQ_OK;
+    if (x_dtype == WQ_BF16) return tq3_mma::encode_bf16(x, n_vec, m, records, nullptr, nullptr, s, true);
+    return tq3_rows::encode(x, x_dtype, n_vec, m, records, nullptr, nullptr, s, true);
+}
+
+extern "C" wq_status tq3_decode_aos(const uint8_t *records, int64_t n_vec, const uint32_t *sign_mask, void *out,
+                                    int out_dtype, void *stream) {
+    if (n_vec < 0) return WQ_ERR_SHAPE;
+    if (!valid_dtype(out_dtype)) return WQ_ERR_DTYPE;
+    if (n_vec == 0) return WQ_OK;
+    if (!records || !sign_mask || !out) return WQ_ERR_NULL;
+    if (n_vec > ((int64_t)1 << 40)) return WQ_ERR_SHAPE;
+    if (!aligned(records, 8) || !aligned(out, 16)) return WQ_ERR_ALIGN;
+    tq3::SignMask m;
+    for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
+    return tq3_rows::decode(records, nullptr, nullptr, n_vec, m, out, out_dtype, static_cast<cudaStream_t>(stream),
+                            true);
 }
 
 extern "C" int64_t tq3_compressed_bytes(int64_t n_vec) {

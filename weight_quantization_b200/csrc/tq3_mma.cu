@@ -192,7 +192,9 @@ constexpr BTable make_default_b() {
 }
 __device__ __align__(128) const BTable kDefaultB = make_default_b();
 
-template <bool kFold>
+// kAoS: 56-byte records (the 48 packed bytes, the norm, the scale) at `packed`; norms and scales
+// are unused.
+template <bool kFold, bool kAoS = false>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_mma(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, SignMask mask, uint8_t *__restrict__ packed,
                float *__restrict__ norms, float *__restrict__ scales) {
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // pass 2: the indices, 32 columns at a time, the reads alternating as in pass 1
         const int64_t v = (stream + it * n_streams) * kTile + tid;
-        uint8_t *const rec = packed + v * 48;
+        uint8_t *const rec = packed + v * (kAoS ? 56 : 48);
         uint32_t o[12];
         tmem_wait(za);
         tmem_ld32(my_lanes + 32, zb);
@@ -365,11 +367,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_mma(it + 1);
         bucket_piece(zb, Mb, K0, K1, K2, o[9], o[10], o[11]);
         if (v < n_vec) {
-            st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
-            st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
-            st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));
-            norms[v] = nrm;
-            scales[v] = scale;
+            if constexpr (kAoS) {  // a 56-byte record is 8-byte aligned
+#pragma unroll
+                for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
+                st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+            } else {
+                st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
+                st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
+                st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));
+                norms[v] = nrm;
+                scales[v] = scale;
+            }
         }
     }
     if (fault && (tid & 31) == 0) atomicOr(&g_fault, 8u);
@@ -418,16 +426,22 @@ wq_status launch(K k, int64_t cnt, const CUtensorMap &tm, const SignMask &m, uin
 }  // namespace
 
 wq_status encode_bf16(const void *x, int64_t n_vec, const SignMask &m, uint8_t *packed, float *norms, float *scales,
-                      cudaStream_t s) {
+                      cudaStream_t s, bool aos) {
     const bool def = tq3::is_default(m);
+    const int64_t rb = aos ? 56 : 48;
     for (int64_t off = 0; off < n_vec; off += tq3::kMaxChunk) {
         const int64_t cnt = n_vec - off < tq3::kMaxChunk ? n_vec - off : tq3::kMaxChunk;
         const unsigned char *xc = static_cast<const unsigned char *>(x) + off * (tq3::kD * 2);
         CUtensorMap tm;
         if (!make_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xc, tq3::kD, (uint64_t)cnt, tq3::kD * 2, 64, kTile))
             return WQ_ERR_CUDA;
-        const wq_status st = def ? launch(encode_mma<true>, cnt, tm, m, packed + off * 48, norms + off, scales + off, s)
-                                 : launch(encode_mma<false>, cnt, tm, m, packed + off * 48, norms + off, scales + off, s);
+        uint8_t *const pc = packed + off * rb;
+        float *const nc = aos ? nullptr : norms + off;
+        float *const sc = aos ? nullptr : scales + off;
+        const wq_status st = aos ? (def ? launch(encode_mma<true, true>, cnt, tm, m, pc, nc, sc, s)
+                                        : launch(encode_mma<false, true>, cnt, tm, m, pc, nc, sc, s))
+                                 : (def ? launch(encode_mma<true>, cnt, tm, m, pc, nc, sc, s)
+                                        : launch(encode_mma<false>, cnt, tm, m, pc, nc, sc, s));
         if (st != WQ_OK) return st;
     }
     return WQ_OK;

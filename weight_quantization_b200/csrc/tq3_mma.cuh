@@ -11,9 +11,10 @@
 namespace wq {
 namespace tq3_mma {
 
-// tq3_quantize of n_vec bf16 vectors (same contract and precision as the fast TQ3 encoder).
+// tq3_quantize of n_vec bf16 vectors (same contract and precision as the fast TQ3 encoder). With
+// aos, `packed` receives 56-byte records (packed bytes, norm, scale) and norms/scales are unused.
 wq_status encode_bf16(const void *x, int64_t n_vec, const tq3::SignMask &m, uint8_t *packed, float *norms,
-                      float *scales, cudaStream_t s);
+                      float *scales, cudaStream_t s, bool aos = false);
 
 // Reads and clears the fault bits of this kernel (bit 3: a bounded wait for a TMA tile or for the
 // tensor-core product ran out).

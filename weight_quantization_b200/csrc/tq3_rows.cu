@@ -108,7 +108,9 @@ struct EncGeo {
 // The positive TQ3_BOUNDARIES (fp32); the others are their negatives and 0.
 __device__ __forceinline__ float edge(int k) { return k == 0 ? 0.2304f : k == 1 ? 0.4824f : 0.7992f; }
 
-template <bool kBf16, bool kFold>
+// kAoS: 56-byte records (the 48 packed bytes, the norm, the scale) at `packed`; norms and scales
+// are unused (here and in decode_rows).
+template <bool kBf16, bool kFold, bool kAoS = false>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
     encode_rows(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, SignMask mask, uint8_t *__restrict__ packed,
                 float *__restrict__ norms, float *__restrict__ scales) {
@@ -314,12 +316,19 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
                 o[3 * q + 1] = (g[4 * q + 1] >> 8) | (g[4 * q + 2] << 16);
                 o[3 * q + 2] = (g[4 * q + 2] >> 16) | (g[4 * q + 3] << 8);
             }
-            uint8_t *rec = packed + v * 48;
-            st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
-            st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
-            st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));
-            norms[v] = nrm;
-            scales[v] = scale;
+            if constexpr (kAoS) {  // a 56-byte record is 8-byte aligned
+                uint8_t *rec = packed + v * 56;
+#pragma unroll
+                for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
+                st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+            } else {
+                uint8_t *rec = packed + v * 48;
+                st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
+                st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
+                st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));
+                norms[v] = nrm;
+                scales[v] = scale;
+            }
         }
     }
 }
@@ -332,16 +341,29 @@ struct Rec {
     float n, s;
 };
 
+template <bool kAoS>
 __device__ __forceinline__ Rec load_rec(const uint8_t *__restrict__ packed, const float *__restrict__ norms,
                                         const float *__restrict__ scales, int64_t n_vec, int64_t v) {
     Rec r;
     if (v < n_vec) {
-        const uint8_t *p = packed + v * 48;
-        r.q[0] = ld_nc16(p);
-        r.q[1] = ld_nc16(p + 16);
-        r.q[2] = ld_nc16(p + 32);
-        r.n = __ldg(norms + v);
-        r.s = __ldg(scales + v);
+        if constexpr (kAoS) {  // a 56-byte record is 8-byte aligned
+            const uint8_t *p = packed + v * 56;
+            uint2 w[7];
+#pragma unroll
+            for (int q = 0; q < 7; ++q) w[q] = __ldg(reinterpret_cast<const uint2 *>(p) + q);
+            r.q[0] = make_uint4(w[0].x, w[0].y, w[1].x, w[1].y);
+            r.q[1] = make_uint4(w[2].x, w[2].y, w[3].x, w[3].y);
+            r.q[2] = make_uint4(w[4].x, w[4].y, w[5].x, w[5].y);
+            r.n = __uint_as_float(w[6].x);
+            r.s = __uint_as_float(w[6].y);
+        } else {
+            const uint8_t *p = packed + v * 48;
+            r.q[0] = ld_nc16(p);
+            r.q[1] = ld_nc16(p + 16);
+            r.q[2] = ld_nc16(p + 32);
+            r.n = __ldg(norms + v);
+            r.s = __ldg(scales + v);
+        }
     } else {
         r.q[0] = r.q[1] = r.q[2] = make_uint4(0u, 0u, 0u, 0u);
         r.n = r.s = 0.0f;
@@ -357,7 +379,7 @@ struct DecGeo {
     static constexpr int kSmem = 1024 + kBufs * kTileBytes;
 };
 
-template <bool kBf16Out, bool kFold>
+template <bool kBf16Out, bool kFold, bool kAoS = false>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
     decode_rows(const uint8_t *__restrict__ packed, const float *__restrict__ norms, const float *__restrict__ scales,
                 int64_t n_vec, SignMask mask, const __grid_constant__ CUtensorMap omap) {
@@ -375,21 +397,25 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
     const bool pf_ok = ((reinterpret_cast<uintptr_t>(packed) | reinterpret_cast<uintptr_t>(norms) |
                          reinterpret_cast<uintptr_t>(scales)) & 15) == 0;
     pdl_wait();  // the records may come from the kernel before this one
-    Rec cur = load_rec(packed, norms, scales, n_vec, tile * kTile + tid);
+    Rec cur = load_rec<kAoS>(packed, norms, scales, n_vec, tile * kTile + tid);
     for (int it = 0; tile < n_tiles; ++it, tile += gridDim.x) {
         // on its last tile the block lets the next kernel in the stream be scheduled: its set-up
         // overlaps this kernel's tail (it still waits for this kernel to finish before reading)
         if (tile + gridDim.x >= n_tiles) pdl_trigger();
-        const Rec nxt = load_rec(packed, norms, scales, n_vec, (tile + gridDim.x) * kTile + tid);
+        const Rec nxt = load_rec<kAoS>(packed, norms, scales, n_vec, (tile + gridDim.x) * kTile + tid);
         // the records of the tile after that go into L2 now, so next iteration's load finds them
         // there (whole 16-byte units inside the arrays only)
         if (tid == 0 && pf_ok && tile + 2 * gridDim.x < n_tiles) {
             const int64_t v0 = (tile + 2 * gridDim.x) * kTile;
             const int64_t cnt = (n_vec - v0 < kTile ? n_vec - v0 : kTile) & ~int64_t(3);
             if (cnt > 0) {
-                bulk_prefetch_l2(packed + v0 * 48, (uint32_t)(cnt * 48));
-                bulk_prefetch_l2(norms + v0, (uint32_t)(cnt * 4));
-                bulk_prefetch_l2(scales + v0, (uint32_t)(cnt * 4));
+                if constexpr (kAoS) {
+                    bulk_prefetch_l2(packed + v0 * 56, (uint32_t)(cnt * 56));
+                } else {
+                    bulk_prefetch_l2(packed + v0 * 48, (uint32_t)(cnt * 48));
+                    bulk_prefetch_l2(norms + v0, (uint32_t)(cnt * 4));
+                    bulk_prefetch_l2(scales + v0, (uint32_t)(cnt * 4));
+                }
             }
         }
         unsigned char *buf = obuf + (it % G::kBufs) * G::kTileBytes;
@@ -524,7 +550,7 @@ wq_status launch_enc(K k, size_t smem, int64_t cnt, const CUtensorMap &tm, const
 }
 
 wq_status encode(const void *x, int x_dtype, int64_t n_vec, const SignMask &m, uint8_t *packed, float *norms,
-                 float *scales, cudaStream_t s) {
+                 float *scales, cudaStream_t s, bool aos) {
     const bool def = tq3::is_default(m), bf = x_dtype == WQ_BF16;
     const int esz = bf ? 2 : 4;
     const size_t smem = bf ? EncGeo<true>::kSmem : EncGeo<false>::kSmem;
@@ -535,10 +561,15 @@ wq_status encode(const void *x, int x_dtype, int64_t n_vec, const SignMask &m, u
         if (!make_tmap_2d(&tm, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, xc, tq3::kD,
                           (uint64_t)cnt, tq3::kD * esz, bf ? 64 : 32, kTile))
             return WQ_ERR_CUDA;
-        uint8_t *pc = packed + off * 48;
-        float *nc = norms + off, *sc = scales + off;
+        uint8_t *pc = packed + off * (aos ? 56 : 48);
+        float *nc = aos ? nullptr : norms + off, *sc = aos ? nullptr : scales + off;
         wq_status st;
-        if (bf && def)
+        if (aos)
+            st = bf ? (def ? launch_enc(encode_rows<true, true, true>, smem, cnt, tm, m, pc, nc, sc, s)
+                           : launch_enc(encode_rows<true, false, true>, smem, cnt, tm, m, pc, nc, sc, s))
+                    : (def ? launch_enc(encode_rows<false, true, true>, smem, cnt, tm, m, pc, nc, sc, s)
+                           : launch_enc(encode_rows<false, false, true>, smem, cnt, tm, m, pc, nc, sc, s));
+        else if (bf && def)
             st = launch_enc(encode_rows<true, true>, smem, cnt, tm, m, pc, nc, sc, s);
         else if (bf)
             st = launch_enc(encode_rows<true, false>, smem, cnt, tm, m, pc, nc, sc, s);
@@ -561,7 +592,7 @@ wq_status launch_dec(K k, size_t smem, const uint8_t *pc, const float *nc, const
 }
 
 wq_status decode(const uint8_t *packed, const float *norms, const float *scales, int64_t n_vec, const SignMask &m,
-                 void *out, int out_dtype, cudaStream_t s) {
+                 void *out, int out_dtype, cudaStream_t s, bool aos) {
     const bool def = tq3::is_default(m), bf = out_dtype == WQ_BF16;
     const int esz = bf ? 2 : 4;
     const size_t smem = bf ? DecGeo<true>::kSmem : DecGeo<false>::kSmem;
@@ -572,10 +603,15 @@ wq_status decode(const uint8_t *packed, const float *norms, const float *scales,
         if (!make_tmap_2d(&tm, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, oc, tq3::kD,
                           (uint64_t)cnt, tq3::kD * esz, bf ? 64 : 32, kTile))
             return WQ_ERR_CUDA;
-        const uint8_t *pc = packed + off * 48;
-        const float *nc = norms + off, *sc = scales + off;
+        const uint8_t *pc = packed + off * (aos ? 56 : 48);
+        const float *nc = aos ? nullptr : norms + off, *sc = aos ? nullptr : scales + off;
         wq_status st;
-        if (bf && def)
+        if (aos)
+            st = bf ? (def ? launch_dec(decode_rows<true, true, true>, smem, pc, nc, sc, cnt, m, tm, s)
+                           : launch_dec(decode_rows<true, false, true>, smem, pc, nc, sc, cnt, m, tm, s))
+                    : (def ? launch_dec(decode_rows<false, true, true>, smem, pc, nc, sc, cnt, m, tm, s)
+                           : launch_dec(decode_rows<false, false, true>, smem, pc, nc, sc, cnt, m, tm, s));
+        else if (bf && def)
             st = launch_dec(decode_rows<true, true>, smem, pc, nc, sc, cnt, m, tm, s);
         else if (bf)
             st = launch_dec(decode_rows<true, false>, smem, pc, nc, sc, cnt, m, tm, s);

@@ -25,6 +25,8 @@ PROTOTYPES = {
     "tq3_encode": (_int, [_vp, _int, _i64, _vp, _vp, _vp, _vp, _vp]),
     "tq3_encode_exact": (_int, [_vp, _int, _i64, _vp, _vp, _vp, _vp, _vp]),
     "tq3_decode": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _int, _vp]),
+    "tq3_encode_aos": (_int, [_vp, _int, _i64, _vp, _vp, _vp]),
+    "tq3_decode_aos": (_int, [_vp, _i64, _vp, _vp, _int, _vp]),
     "tq3_compressed_bytes": (_i64, [_i64]),
     "rpbh_quantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp]),
     "rpbh_dequantize_weight": (_int, [_vp, _vp, _int, _i64, _i64, _int, _vp, _vp, _vp, _int, _vp, _int, _vp]),
@@ -134,6 +136,37 @@ def tq3_decode(packed: torch.Tensor, norms: torch.Tensor, scales: torch.Tensor, 
     st = lib().tq3_decode(_dev(packed, "packed"), _dev(norms, "norms"), _dev(scales, "scales"), n_vec,
                           m.ctypes.data, _dev(out, "out"), _DT[out.dtype], _stream(packed.device))
     _check("tq3_decode", st)
+    return out
+
+
+def tq3_encode_aos(x: torch.Tensor, sign_mask, records=None):
+    """TQ3-encode a [..., D] fp32/bf16 CUDA tensor into 56-byte records [..., D/128, 56] (the packed
+    bytes, the fp32 norm, the fp32 scale)."""
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32 or bfloat16")
+    if x.ndim == 0 or x.shape[-1] % 128 != 0 or x.shape[-1] <= 0:
+        raise ValueError("last dim must be a positive multiple of 128")
+    lead = tuple(x.shape[:-1]) + (x.shape[-1] // 128,)
+    if records is None:
+        records = torch.empty(lead + (56,), dtype=torch.uint8, device=x.device)
+    m = _mask_arg(sign_mask)
+    st = lib().tq3_encode_aos(_dev(x, "x"), _DT[x.dtype], x.numel() // 128, m.ctypes.data, _dev(records, "records"),
+                              _stream(x.device))
+    _check("tq3_encode_aos", st)
+    return records
+
+
+def tq3_decode_aos(records: torch.Tensor, sign_mask, out_dtype=torch.float32, out=None):
+    """Decode 56-byte TQ3 records [..., 56] back to [..., 128] values of out_dtype (fp32 or bf16)."""
+    if records.shape[-1] != 56:
+        raise ValueError("records must be [..., 56]")
+    n_vec = records.numel() // 56
+    if out is None:
+        out = torch.empty(tuple(records.shape[:-1]) + (128,), dtype=out_dtype, device=records.device)
+    m = _mask_arg(sign_mask)
+    st = lib().tq3_decode_aos(_dev(records, "records"), n_vec, m.ctypes.data, _dev(out, "out"), _DT[out.dtype],
+                              _stream(records.device))
+    _check("tq3_decode_aos", st)
     return out
 
 
