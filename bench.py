@@ -195,8 +195,18 @@ class KVWorkload:
         self.out = [torch.empty(n, 128, dtype=torch.bfloat16, device=dev)]
         for k in range(R):
             self._encode(k)
+        # 56-byte records (timed beside the step), rotating over R sets as well; the paged forms
+        # use pages of 16 records in a random page order
+        self.recs = [ops.tq3_encode_aos(self.x[0], self.mask).view(n, 56) for _ in range(R)]
+        self.page = 16
+        g = torch.Generator().manual_seed(seed)
+        self.table = torch.randperm(n // self.page, generator=g).to(torch.int32).to(dev)
+        pos = torch.arange(n, dtype=torch.int64)
+        self.slots = (self.table.cpu().to(torch.int64)[pos // self.page] * self.page + pos % self.page).to(dev)
         self.kernels = ["tq3_encode", "tq3_decode"]
-        self.bytes_per_launch = {"tq3_encode": 312 * n, "tq3_decode": 312 * n}
+        self.bytes_per_launch = {"tq3_encode": 312 * n, "tq3_decode": 312 * n, "tq3_encode_aos": 312 * n,
+                                 "tq3_decode_aos": 312 * n, "tq3_encode_slots": 320 * n,
+                                 "tq3_decode_paged": (312 + 4 / self.page) * n}
         self.l2 = (f"cache (134 MB) larger than L2; records rotate over {R} sets: launch k encodes into "
                    f"set k % {R} and decodes set (k + 1) % {R}, written {R - 1} launches earlier")
 
@@ -218,8 +228,18 @@ class KVWorkload:
         return [("tq3_encode", 1, self._encode), ("tq3_decode", 1, self._decode)]
 
     def extras(self):
-        """Kernels timed beside the step (not part of it): the bit-exact encoder on the same cache."""
-        return [("tq3_encode_exact", 1, lambda k: self._encode(k, exact=True))]
+        """Kernels timed beside the step (not part of it): the bit-exact encoder on the same cache and
+        the codec on 56-byte records."""
+        o, R = self.ops, self.RSETS
+        return [("tq3_encode_exact", 1, lambda k: self._encode(k, exact=True)),
+                ("tq3_encode_aos", 1, lambda k: o.tq3_encode_aos(self.x[0], self.mask, records=self.recs[k % R])),
+                ("tq3_decode_aos", 1, lambda k: o.tq3_decode_aos(self.recs[(k + 1) % R], self.mask,
+                                                                 out_dtype=torch.bfloat16, out=self.out[0])),
+                ("tq3_encode_slots", 1, lambda k: o.tq3_encode_slots(self.x[0], self.mask, self.slots,
+                                                                     self.recs[k % R])),
+                ("tq3_decode_paged", 1, lambda k: o.tq3_decode_paged(self.recs[(k + 1) % R], self.table, self.page,
+                                                                     self.units, self.mask, out_dtype=torch.bfloat16,
+                                                                     out=self.out[0]))]
 
     def step(self, k=0):
         for _, _, fn in self.parts():

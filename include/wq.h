@@ -107,6 +107,29 @@ wq_status tq3_encode_aos(const void *x, int x_dtype, int64_t n_vec, const uint32
 wq_status tq3_decode_aos(const uint8_t *records, int64_t n_vec, const uint32_t *sign_mask, void *out,
                          int out_dtype, void *stream);
 
+/* tq3_encode_slots / tq3_decode_paged -- the same codec on a KV cache kept as a pool of 56-byte
+ * records (the record of tq3_encode_aos) that is written and read through indirection, as a paged
+ * cache is: appended vectors are scattered to free slots, and a sequence is read back through its
+ * page table. No counterpart on the page beyond the record itself; the arithmetic is that of
+ * tq3_encode_aos / tq3_decode_aos, record by record.
+ * tq3_encode_slots: vector v of x goes to record slots[v] of the pool.
+ *   slots      device, n_vec x int64, 8-byte aligned. A negative slot skips the vector (padding);
+ *              a slot >= n_pool is skipped and sets device fault bit 6. Two vectors with the same
+ *              slot race (one of them is stored).
+ *   pool       device, n_pool x 56 bytes, 8-byte aligned; records not named by a slot are untouched.
+ * tq3_decode_paged: out[p] = decode(record page_table[p / page_size] * page_size + p % page_size)
+ * for p = 0 .. n_vec-1.
+ *   page_table device, n_pages x int32, 4-byte aligned; n_vec <= n_pages * page_size (else
+ *              WQ_ERR_SHAPE). A negative entry, or one whose record lies at or beyond n_pool,
+ *              decodes as zeros and sets device fault bit 6.
+ *   page_size  a power of two, 1 .. 2^30 (else WQ_ERR_SHAPE).
+ *   out        device, n_vec x 128 elements of out_dtype, 16-byte aligned. */
+wq_status tq3_encode_slots(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
+                           const int64_t *slots, uint8_t *pool, int64_t n_pool, void *stream);
+wq_status tq3_decode_paged(const uint8_t *pool, int64_t n_pool, const int32_t *page_table, int64_t n_pages,
+                           int64_t page_size, int64_t n_vec, const uint32_t *sign_mask, void *out,
+                           int out_dtype, void *stream);
+
 /* tq3_compressed_bytes -- tq3_memory_bytes' compressed size for n_vec vectors: 56 * n_vec
  * (-1 if n_vec < 0 or the product overflows). */
 int64_t tq3_compressed_bytes(int64_t n_vec);
@@ -210,7 +233,9 @@ wq_status wq_rpbh_codebook(int bits, int64_t d, float *out);
  * leaving its outputs unspecified: bit 0 a TQ3 kernel waiting for a TMA tile, bit 1 an RPBH kernel
  * waiting for a row copy, bit 3 the tensor-core TQ3 encoder waiting for a tile or its product,
  * bit 4 rpbh_linear waiting for a tile, the unpacked weights or its product, bit 5 the self-test
- * wq_selftest_wait_timeout.
+ * wq_selftest_wait_timeout. Bit 6 is not a wait: tq3_encode_slots or tq3_decode_paged met a slot or
+ * page-table entry outside the pool (that record was skipped, or decoded as zeros; the rest of the
+ * call is complete).
  * Synchronous (a device-to-host copy on the legacy default stream); `flags` is host memory.
  * Errors: WQ_ERR_NULL, WQ_ERR_CUDA. */
 wq_status wq_device_fault(unsigned int *flags);

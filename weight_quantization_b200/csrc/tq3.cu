@@ -353,8 +353,8 @@ extern "C" wq_status tq3_encode_aos(const void *x, int x_dtype, int64_t n_vec, c
     tq3::SignMask m;
     for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (x_dtype == WQ_BF16) return tq3_mma::encode_bf16(x, n_vec, m, records, nullptr, nullptr, s, true);
-    return tq3_rows::encode(x, x_dtype, n_vec, m, records, nullptr, nullptr, s, true);
+    if (x_dtype == WQ_BF16) return tq3_mma::encode_bf16(x, n_vec, m, records, nullptr, nullptr, s, tq3::kAoS);
+    return tq3_rows::encode(x, x_dtype, n_vec, m, records, nullptr, nullptr, s, tq3::kAoS);
 }
 
 extern "C" wq_status tq3_decode_aos(const uint8_t *records, int64_t n_vec, const uint32_t *sign_mask, void *out,
@@ -368,7 +368,43 @@ extern "C" wq_status tq3_decode_aos(const uint8_t *records, int64_t n_vec, const
     tq3::SignMask m;
     for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
     return tq3_rows::decode(records, nullptr, nullptr, n_vec, m, out, out_dtype, static_cast<cudaStream_t>(stream),
-                            true);
+                            tq3::kAoS);
+}
+
+extern "C" wq_status tq3_encode_slots(const void *x, int x_dtype, int64_t n_vec, const uint32_t *sign_mask,
+                                      const int64_t *slots, uint8_t *pool, int64_t n_pool, void *stream) {
+    if (n_vec < 0 || n_pool < 0) return WQ_ERR_SHAPE;
+    if (!valid_dtype(x_dtype)) return WQ_ERR_DTYPE;
+    if (n_vec == 0) return WQ_OK;
+    if (!x || !sign_mask || !slots || !pool) return WQ_ERR_NULL;
+    if (n_vec > ((int64_t)1 << 40) || n_pool > ((int64_t)1 << 40)) return WQ_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(pool, 8) || !aligned(slots, 8)) return WQ_ERR_ALIGN;
+    tq3::SignMask m;
+    for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
+    const tq3::PoolMap pm{slots, 0, n_pool, 0};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (x_dtype == WQ_BF16) return tq3_mma::encode_bf16(x, n_vec, m, pool, nullptr, nullptr, s, tq3::kPool, pm);
+    return tq3_rows::encode(x, x_dtype, n_vec, m, pool, nullptr, nullptr, s, tq3::kPool, pm);
+}
+
+extern "C" wq_status tq3_decode_paged(const uint8_t *pool, int64_t n_pool, const int32_t *page_table,
+                                      int64_t n_pages, int64_t page_size, int64_t n_vec, const uint32_t *sign_mask,
+                                      void *out, int out_dtype, void *stream) {
+    if (n_vec < 0 || n_pool < 0 || n_pages < 0) return WQ_ERR_SHAPE;
+    if (page_size < 1 || page_size > ((int64_t)1 << 30) || (page_size & (page_size - 1))) return WQ_ERR_SHAPE;
+    if (!valid_dtype(out_dtype)) return WQ_ERR_DTYPE;
+    if (n_vec == 0) return WQ_OK;
+    if (!pool || !page_table || !sign_mask || !out) return WQ_ERR_NULL;
+    if (n_vec > ((int64_t)1 << 40) || n_pool > ((int64_t)1 << 40) || n_pages > ((int64_t)1 << 40)) return WQ_ERR_SHAPE;
+    if (n_vec > n_pages * page_size) return WQ_ERR_SHAPE;  // the table must cover every vector read
+    if (!aligned(pool, 8) || !aligned(page_table, 4) || !aligned(out, 16)) return WQ_ERR_ALIGN;
+    tq3::SignMask m;
+    for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
+    int shift = 0;
+    while ((int64_t(1) << shift) < page_size) ++shift;
+    const tq3::PoolMap pm{page_table, 0, n_pool, shift};
+    return tq3_rows::decode(pool, nullptr, nullptr, n_vec, m, out, out_dtype, static_cast<cudaStream_t>(stream),
+                            tq3::kPool, pm);
 }
 
 extern "C" int64_t tq3_compressed_bytes(int64_t n_vec) {

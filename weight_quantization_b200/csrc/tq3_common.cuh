@@ -15,6 +15,24 @@ struct SignMask {
     uint32_t w[4];  // bit i = sign draw i (1 -> +1, 0 -> -1)
 };
 
+// Where a launch's records live. kSoA: three arrays, packed[n][48], norms[n], scales[n]. kAoS:
+// 56-byte records (the 48 packed bytes, the fp32 norm, the fp32 scale) at byte 56 v. kPool:
+// 56-byte records in a pool, placed through an index: an int64 slot per vector when writing
+// (negative: the vector is not stored), an int32 page table when reading (logical vector p lives in
+// record table[p >> shift] * 2^shift + (p mod 2^shift)).
+enum Layout : int { kSoA = 0, kAoS = 1, kPool = 2 };
+
+struct PoolMap {
+    const void *index;  // int64 slots (encode) or int32 page table (decode); unused for kSoA, kAoS
+    int64_t v0;         // logical position of the launch's first vector (decode)
+    int64_t n_pool;     // records in the pool
+    int shift;          // log2 of the page size (decode)
+};
+
+// Fault bit set by a kernel that met a slot or page-table entry outside the pool (the record was
+// not written, or was decoded as zeros).
+constexpr unsigned int kFaultPoolIndex = 64u;
+
 // The draws of _generate_sign_flips(128, seed=42): the page's fixed table. Kernels specialised on it
 // fold the flips into compile-time constants; any other table takes the runtime path.
 __host__ __device__ constexpr uint32_t default_mask_word(int w) {

@@ -192,12 +192,13 @@ constexpr BTable make_default_b() {
 }
 __device__ __align__(128) const BTable kDefaultB = make_default_b();
 
-// kAoS: 56-byte records (the 48 packed bytes, the norm, the scale) at `packed`; norms and scales
-// are unused.
-template <bool kFold, bool kAoS = false>
+// kLay (tq3::Layout): kSoA writes packed, norms and scales; kAoS writes 56-byte records (the 48
+// packed bytes, the norm, the scale) at `packed`; kPool writes record v to slot pm.index[v] of the
+// pool at `packed` (a negative slot: not stored). Norms and scales are unused for the record layouts.
+template <bool kFold, int kLay = tq3::kSoA>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_mma(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, SignMask mask, uint8_t *__restrict__ packed,
-               float *__restrict__ norms, float *__restrict__ scales) {
+               float *__restrict__ norms, float *__restrict__ scales, tq3::PoolMap pm) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *const base = tq3::tile_base(smem_raw);
     const int grp = threadIdx.x >> 7, tid = threadIdx.x & 127, warp = tid >> 5;
@@ -348,7 +349,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // pass 2: the indices, 32 columns at a time, the reads alternating as in pass 1
         const int64_t v = (stream + it * n_streams) * kTile + tid;
-        uint8_t *const rec = packed + v * (kAoS ? 56 : 48);
+        int64_t slot = v;  // the slot's load is issued here, ahead of its use at the store
+        if constexpr (kLay == tq3::kPool) slot = v < n_vec ? __ldg(static_cast<const int64_t *>(pm.index) + v) : -1;
+        uint8_t *const rec = packed + slot * (kLay == tq3::kSoA ? 48 : 56);
         uint32_t o[12];
         tmem_wait(za);
         tmem_ld32(my_lanes + 32, zb);
@@ -367,10 +370,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_mma(it + 1);
         bucket_piece(zb, Mb, K0, K1, K2, o[9], o[10], o[11]);
         if (v < n_vec) {
-            if constexpr (kAoS) {  // a 56-byte record is 8-byte aligned
+            if constexpr (kLay != tq3::kSoA) {  // a 56-byte record is 8-byte aligned
+                if (kLay == tq3::kPool && slot >= pm.n_pool) atomicOr(&g_fault, tq3::kFaultPoolIndex);
+                if (kLay == tq3::kAoS || (slot >= 0 && slot < pm.n_pool)) {
 #pragma unroll
-                for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
-                st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+                    for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
+                    st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+                }
             } else {
                 st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
                 st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
@@ -410,14 +416,14 @@ int sm_count() {
 
 template <typename K>
 wq_status launch(K k, int64_t cnt, const CUtensorMap &tm, const SignMask &m, uint8_t *pc, float *nc, float *sc,
-                 cudaStream_t s) {
+                 const tq3::PoolMap &pm, cudaStream_t s) {
     if (!ensure_dynamic_smem(reinterpret_cast<const void *>(k), kSmem)) return WQ_ERR_CUDA;
     // one CTA per SM (it holds all 512 tensor-memory columns), never more CTAs than tile triples
     const int64_t tiles = (cnt + kTile - 1) / kTile;
     const int64_t triples = (tiles + kGroups - 1) / kGroups;
     const int64_t g_ = sm_count() > 0 ? sm_count() : 1;
     const int64_t g = g_ < triples ? g_ : triples;
-    if (launch_pdl(k, (unsigned)g, kThreads, kSmem, s, cnt, tm, m, pc, nc, sc) != cudaSuccess) {
+    if (launch_pdl(k, (unsigned)g, kThreads, kSmem, s, cnt, tm, m, pc, nc, sc, pm) != cudaSuccess) {
         cudaGetLastError();
         return WQ_ERR_CUDA;
     }
@@ -426,22 +432,29 @@ wq_status launch(K k, int64_t cnt, const CUtensorMap &tm, const SignMask &m, uin
 }  // namespace
 
 wq_status encode_bf16(const void *x, int64_t n_vec, const SignMask &m, uint8_t *packed, float *norms, float *scales,
-                      cudaStream_t s, bool aos) {
+                      cudaStream_t s, int layout, const tq3::PoolMap &pool) {
     const bool def = tq3::is_default(m);
-    const int64_t rb = aos ? 56 : 48;
     for (int64_t off = 0; off < n_vec; off += tq3::kMaxChunk) {
         const int64_t cnt = n_vec - off < tq3::kMaxChunk ? n_vec - off : tq3::kMaxChunk;
         const unsigned char *xc = static_cast<const unsigned char *>(x) + off * (tq3::kD * 2);
         CUtensorMap tm;
         if (!make_tmap_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xc, tq3::kD, (uint64_t)cnt, tq3::kD * 2, 64, kTile))
             return WQ_ERR_CUDA;
-        uint8_t *const pc = packed + off * rb;
-        float *const nc = aos ? nullptr : norms + off;
-        float *const sc = aos ? nullptr : scales + off;
-        const wq_status st = aos ? (def ? launch(encode_mma<true, true>, cnt, tm, m, pc, nc, sc, s)
-                                        : launch(encode_mma<false, true>, cnt, tm, m, pc, nc, sc, s))
-                                 : (def ? launch(encode_mma<true>, cnt, tm, m, pc, nc, sc, s)
-                                        : launch(encode_mma<false>, cnt, tm, m, pc, nc, sc, s));
+        wq_status st;
+        if (layout == tq3::kPool) {  // the pool is not offset; the chunk's slots are
+            tq3::PoolMap pm = pool;
+            pm.index = static_cast<const int64_t *>(pool.index) + off;
+            st = def ? launch(encode_mma<true, tq3::kPool>, cnt, tm, m, packed, nullptr, nullptr, pm, s)
+                     : launch(encode_mma<false, tq3::kPool>, cnt, tm, m, packed, nullptr, nullptr, pm, s);
+        } else if (layout == tq3::kAoS) {
+            uint8_t *const pc = packed + off * 56;
+            st = def ? launch(encode_mma<true, tq3::kAoS>, cnt, tm, m, pc, nullptr, nullptr, pool, s)
+                     : launch(encode_mma<false, tq3::kAoS>, cnt, tm, m, pc, nullptr, nullptr, pool, s);
+        } else {
+            uint8_t *const pc = packed + off * 48;
+            st = def ? launch(encode_mma<true>, cnt, tm, m, pc, norms + off, scales + off, pool, s)
+                     : launch(encode_mma<false>, cnt, tm, m, pc, norms + off, scales + off, pool, s);
+        }
         if (st != WQ_OK) return st;
     }
     return WQ_OK;

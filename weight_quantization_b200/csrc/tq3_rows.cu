@@ -108,12 +108,13 @@ struct EncGeo {
 // The positive TQ3_BOUNDARIES (fp32); the others are their negatives and 0.
 __device__ __forceinline__ float edge(int k) { return k == 0 ? 0.2304f : k == 1 ? 0.4824f : 0.7992f; }
 
-// kAoS: 56-byte records (the 48 packed bytes, the norm, the scale) at `packed`; norms and scales
-// are unused (here and in decode_rows).
-template <bool kBf16, bool kFold, bool kAoS = false>
+// kLay (tq3::Layout): kSoA writes packed, norms and scales; kAoS writes 56-byte records at
+// `packed`; kPool writes record v to slot pm.index[v] of the pool at `packed` (here and in
+// decode_rows, norms and scales are unused for the record layouts).
+template <bool kBf16, bool kFold, int kLay = tq3::kSoA>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
     encode_rows(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, SignMask mask, uint8_t *__restrict__ packed,
-                float *__restrict__ norms, float *__restrict__ scales) {
+                float *__restrict__ norms, float *__restrict__ scales, tq3::PoolMap pm) {
     using G = EncGeo<kBf16>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *const base = tq3::tile_base(smem_raw);
@@ -300,6 +301,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         }
         const int64_t v = (blockIdx.x + it * gridDim.x) * kTile + tid;
         if (v < n_vec) {
+            int64_t slot = v;
+            if constexpr (kLay == tq3::kPool) slot = __ldg(static_cast<const int64_t *>(pm.index) + v);
             uint32_t g[16];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -316,11 +319,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
                 o[3 * q + 1] = (g[4 * q + 1] >> 8) | (g[4 * q + 2] << 16);
                 o[3 * q + 2] = (g[4 * q + 2] >> 16) | (g[4 * q + 3] << 8);
             }
-            if constexpr (kAoS) {  // a 56-byte record is 8-byte aligned
-                uint8_t *rec = packed + v * 56;
+            if constexpr (kLay != tq3::kSoA) {  // a 56-byte record is 8-byte aligned
+                if (kLay == tq3::kPool && slot >= pm.n_pool) atomicOr(&g_fault, tq3::kFaultPoolIndex);
+                if (kLay == tq3::kAoS || (slot >= 0 && slot < pm.n_pool)) {
+                    uint8_t *rec = packed + slot * 56;
 #pragma unroll
-                for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
-                st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+                    for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
+                    st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+                }
             } else {
                 uint8_t *rec = packed + v * 48;
                 st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
@@ -341,13 +347,30 @@ struct Rec {
     float n, s;
 };
 
-template <bool kAoS>
+// Record of logical vector p (launch-relative) through the page table, or -1 (and the fault bit)
+// for an entry outside the pool.
+__device__ __forceinline__ int64_t pool_record(const tq3::PoolMap &pm, int64_t p) {
+    const int64_t lp = pm.v0 + p;
+    const int32_t page = __ldg(static_cast<const int32_t *>(pm.index) + (lp >> pm.shift));
+    const int64_t r = ((int64_t)page << pm.shift) | (lp & ((int64_t(1) << pm.shift) - 1));
+    if (page < 0 || r >= pm.n_pool) {
+        atomicOr(&g_fault, tq3::kFaultPoolIndex);
+        return -1;
+    }
+    return r;
+}
+
+template <int kLay>
 __device__ __forceinline__ Rec load_rec(const uint8_t *__restrict__ packed, const float *__restrict__ norms,
-                                        const float *__restrict__ scales, int64_t n_vec, int64_t v) {
+                                        const float *__restrict__ scales, int64_t n_vec, int64_t v,
+                                        const tq3::PoolMap &pm) {
     Rec r;
-    if (v < n_vec) {
-        if constexpr (kAoS) {  // a 56-byte record is 8-byte aligned
-            const uint8_t *p = packed + v * 56;
+    int64_t at = v < n_vec ? v : -1;
+    if constexpr (kLay == tq3::kPool)
+        if (at >= 0) at = pool_record(pm, v);
+    if (at >= 0) {
+        if constexpr (kLay != tq3::kSoA) {  // a 56-byte record is 8-byte aligned
+            const uint8_t *p = packed + at * 56;
             uint2 w[7];
 #pragma unroll
             for (int q = 0; q < 7; ++q) w[q] = __ldg(reinterpret_cast<const uint2 *>(p) + q);
@@ -379,10 +402,10 @@ struct DecGeo {
     static constexpr int kSmem = 1024 + kBufs * kTileBytes;
 };
 
-template <bool kBf16Out, bool kFold, bool kAoS = false>
+template <bool kBf16Out, bool kFold, int kLay = tq3::kSoA>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
     decode_rows(const uint8_t *__restrict__ packed, const float *__restrict__ norms, const float *__restrict__ scales,
-                int64_t n_vec, SignMask mask, const __grid_constant__ CUtensorMap omap) {
+                int64_t n_vec, SignMask mask, const __grid_constant__ CUtensorMap omap, tq3::PoolMap pm) {
     using G = DecGeo<kBf16Out>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *const obuf = tq3::tile_base(smem_raw);
@@ -397,19 +420,29 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
     const bool pf_ok = ((reinterpret_cast<uintptr_t>(packed) | reinterpret_cast<uintptr_t>(norms) |
                          reinterpret_cast<uintptr_t>(scales)) & 15) == 0;
     pdl_wait();  // the records may come from the kernel before this one
-    Rec cur = load_rec<kAoS>(packed, norms, scales, n_vec, tile * kTile + tid);
+    Rec cur = load_rec<kLay>(packed, norms, scales, n_vec, tile * kTile + tid, pm);
     for (int it = 0; tile < n_tiles; ++it, tile += gridDim.x) {
         // on its last tile the block lets the next kernel in the stream be scheduled: its set-up
         // overlaps this kernel's tail (it still waits for this kernel to finish before reading)
         if (tile + gridDim.x >= n_tiles) pdl_trigger();
-        const Rec nxt = load_rec<kAoS>(packed, norms, scales, n_vec, (tile + gridDim.x) * kTile + tid);
+        const Rec nxt = load_rec<kLay>(packed, norms, scales, n_vec, (tile + gridDim.x) * kTile + tid, pm);
         // the records of the tile after that go into L2 now, so next iteration's load finds them
         // there (whole 16-byte units inside the arrays only)
         if (tid == 0 && pf_ok && tile + 2 * gridDim.x < n_tiles) {
             const int64_t v0 = (tile + 2 * gridDim.x) * kTile;
             const int64_t cnt = (n_vec - v0 < kTile ? n_vec - v0 : kTile) & ~int64_t(3);
             if (cnt > 0) {
-                if constexpr (kAoS) {
+                if constexpr (kLay == tq3::kPool) {
+                    // with pages of 32 records or more a tile lies inside one page, so its records
+                    // are contiguous in the pool (and start on a 16-byte boundary)
+                    if (pm.shift >= 5) {
+                        const int64_t lp = pm.v0 + v0;
+                        const int32_t page = __ldg(static_cast<const int32_t *>(pm.index) + (lp >> pm.shift));
+                        const int64_t r0 = ((int64_t)page << pm.shift) | (lp & ((int64_t(1) << pm.shift) - 1));
+                        if (page >= 0 && r0 + cnt <= pm.n_pool)
+                            bulk_prefetch_l2(packed + r0 * 56, (uint32_t)(cnt * 56));
+                    }
+                } else if constexpr (kLay == tq3::kAoS) {
                     bulk_prefetch_l2(packed + v0 * 56, (uint32_t)(cnt * 56));
                 } else {
                     bulk_prefetch_l2(packed + v0 * 48, (uint32_t)(cnt * 48));
@@ -542,15 +575,25 @@ int grid_for(K k, size_t smem, int64_t tiles) {
 
 template <typename K>
 wq_status launch_enc(K k, size_t smem, int64_t cnt, const CUtensorMap &tm, const SignMask &m, uint8_t *pc, float *nc,
-                     float *sc, cudaStream_t s) {
+                     float *sc, const tq3::PoolMap &pm, cudaStream_t s) {
     if (!ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return WQ_ERR_CUDA;
     const int64_t tiles = (cnt + kTile - 1) / kTile;
-    k<<<grid_for(k, smem, tiles), kThreads, smem, s>>>(cnt, tm, m, pc, nc, sc);
+    k<<<grid_for(k, smem, tiles), kThreads, smem, s>>>(cnt, tm, m, pc, nc, sc, pm);
     return launch_status();
 }
 
+template <int kLay>
+wq_status launch_enc_lay(bool bf, bool def, size_t smem, int64_t cnt, const CUtensorMap &tm, const SignMask &m,
+                         uint8_t *pc, float *nc, float *sc, const tq3::PoolMap &pm, cudaStream_t s) {
+    if (bf)
+        return def ? launch_enc(encode_rows<true, true, kLay>, smem, cnt, tm, m, pc, nc, sc, pm, s)
+                   : launch_enc(encode_rows<true, false, kLay>, smem, cnt, tm, m, pc, nc, sc, pm, s);
+    return def ? launch_enc(encode_rows<false, true, kLay>, smem, cnt, tm, m, pc, nc, sc, pm, s)
+               : launch_enc(encode_rows<false, false, kLay>, smem, cnt, tm, m, pc, nc, sc, pm, s);
+}
+
 wq_status encode(const void *x, int x_dtype, int64_t n_vec, const SignMask &m, uint8_t *packed, float *norms,
-                 float *scales, cudaStream_t s, bool aos) {
+                 float *scales, cudaStream_t s, int layout, const tq3::PoolMap &pool) {
     const bool def = tq3::is_default(m), bf = x_dtype == WQ_BF16;
     const int esz = bf ? 2 : 4;
     const size_t smem = bf ? EncGeo<true>::kSmem : EncGeo<false>::kSmem;
@@ -561,22 +604,17 @@ wq_status encode(const void *x, int x_dtype, int64_t n_vec, const SignMask &m, u
         if (!make_tmap_2d(&tm, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, xc, tq3::kD,
                           (uint64_t)cnt, tq3::kD * esz, bf ? 64 : 32, kTile))
             return WQ_ERR_CUDA;
-        uint8_t *pc = packed + off * (aos ? 56 : 48);
-        float *nc = aos ? nullptr : norms + off, *sc = aos ? nullptr : scales + off;
         wq_status st;
-        if (aos)
-            st = bf ? (def ? launch_enc(encode_rows<true, true, true>, smem, cnt, tm, m, pc, nc, sc, s)
-                           : launch_enc(encode_rows<true, false, true>, smem, cnt, tm, m, pc, nc, sc, s))
-                    : (def ? launch_enc(encode_rows<false, true, true>, smem, cnt, tm, m, pc, nc, sc, s)
-                           : launch_enc(encode_rows<false, false, true>, smem, cnt, tm, m, pc, nc, sc, s));
-        else if (bf && def)
-            st = launch_enc(encode_rows<true, true>, smem, cnt, tm, m, pc, nc, sc, s);
-        else if (bf)
-            st = launch_enc(encode_rows<true, false>, smem, cnt, tm, m, pc, nc, sc, s);
-        else if (def)
-            st = launch_enc(encode_rows<false, true>, smem, cnt, tm, m, pc, nc, sc, s);
-        else
-            st = launch_enc(encode_rows<false, false>, smem, cnt, tm, m, pc, nc, sc, s);
+        if (layout == tq3::kPool) {  // the pool is not offset; the chunk's slots are
+            tq3::PoolMap pm = pool;
+            pm.index = static_cast<const int64_t *>(pool.index) + off;
+            st = launch_enc_lay<tq3::kPool>(bf, def, smem, cnt, tm, m, packed, nullptr, nullptr, pm, s);
+        } else if (layout == tq3::kAoS) {
+            st = launch_enc_lay<tq3::kAoS>(bf, def, smem, cnt, tm, m, packed + off * 56, nullptr, nullptr, pool, s);
+        } else {
+            st = launch_enc_lay<tq3::kSoA>(bf, def, smem, cnt, tm, m, packed + off * 48, norms + off, scales + off,
+                                           pool, s);
+        }
         if (st != WQ_OK) return st;
     }
     return WQ_OK;
@@ -584,15 +622,26 @@ wq_status encode(const void *x, int x_dtype, int64_t n_vec, const SignMask &m, u
 
 template <typename K>
 wq_status launch_dec(K k, size_t smem, const uint8_t *pc, const float *nc, const float *sc, int64_t cnt,
-                     const SignMask &m, const CUtensorMap &tm, cudaStream_t s) {
+                     const SignMask &m, const CUtensorMap &tm, const tq3::PoolMap &pm, cudaStream_t s) {
     if (!ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return WQ_ERR_CUDA;
     const int64_t tiles = (cnt + kTile - 1) / kTile;
-    k<<<grid_for(k, smem, tiles), kThreads, smem, s>>>(pc, nc, sc, cnt, m, tm);
+    k<<<grid_for(k, smem, tiles), kThreads, smem, s>>>(pc, nc, sc, cnt, m, tm, pm);
     return launch_status();
 }
 
+template <int kLay>
+wq_status launch_dec_lay(bool bf, bool def, size_t smem, const uint8_t *pc, const float *nc, const float *sc,
+                         int64_t cnt, const SignMask &m, const CUtensorMap &tm, const tq3::PoolMap &pm,
+                         cudaStream_t s) {
+    if (bf)
+        return def ? launch_dec(decode_rows<true, true, kLay>, smem, pc, nc, sc, cnt, m, tm, pm, s)
+                   : launch_dec(decode_rows<true, false, kLay>, smem, pc, nc, sc, cnt, m, tm, pm, s);
+    return def ? launch_dec(decode_rows<false, true, kLay>, smem, pc, nc, sc, cnt, m, tm, pm, s)
+               : launch_dec(decode_rows<false, false, kLay>, smem, pc, nc, sc, cnt, m, tm, pm, s);
+}
+
 wq_status decode(const uint8_t *packed, const float *norms, const float *scales, int64_t n_vec, const SignMask &m,
-                 void *out, int out_dtype, cudaStream_t s, bool aos) {
+                 void *out, int out_dtype, cudaStream_t s, int layout, const tq3::PoolMap &pool) {
     const bool def = tq3::is_default(m), bf = out_dtype == WQ_BF16;
     const int esz = bf ? 2 : 4;
     const size_t smem = bf ? DecGeo<true>::kSmem : DecGeo<false>::kSmem;
@@ -603,22 +652,17 @@ wq_status decode(const uint8_t *packed, const float *norms, const float *scales,
         if (!make_tmap_2d(&tm, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, oc, tq3::kD,
                           (uint64_t)cnt, tq3::kD * esz, bf ? 64 : 32, kTile))
             return WQ_ERR_CUDA;
-        const uint8_t *pc = packed + off * (aos ? 56 : 48);
-        const float *nc = aos ? nullptr : norms + off, *sc = aos ? nullptr : scales + off;
         wq_status st;
-        if (aos)
-            st = bf ? (def ? launch_dec(decode_rows<true, true, true>, smem, pc, nc, sc, cnt, m, tm, s)
-                           : launch_dec(decode_rows<true, false, true>, smem, pc, nc, sc, cnt, m, tm, s))
-                    : (def ? launch_dec(decode_rows<false, true, true>, smem, pc, nc, sc, cnt, m, tm, s)
-                           : launch_dec(decode_rows<false, false, true>, smem, pc, nc, sc, cnt, m, tm, s));
-        else if (bf && def)
-            st = launch_dec(decode_rows<true, true>, smem, pc, nc, sc, cnt, m, tm, s);
-        else if (bf)
-            st = launch_dec(decode_rows<true, false>, smem, pc, nc, sc, cnt, m, tm, s);
-        else if (def)
-            st = launch_dec(decode_rows<false, true>, smem, pc, nc, sc, cnt, m, tm, s);
-        else
-            st = launch_dec(decode_rows<false, false>, smem, pc, nc, sc, cnt, m, tm, s);
+        if (layout == tq3::kPool) {  // the pool is not offset; the page-table position is
+            tq3::PoolMap pm = pool;
+            pm.v0 = pool.v0 + off;
+            st = launch_dec_lay<tq3::kPool>(bf, def, smem, packed, nullptr, nullptr, cnt, m, tm, pm, s);
+        } else if (layout == tq3::kAoS) {
+            st = launch_dec_lay<tq3::kAoS>(bf, def, smem, packed + off * 56, nullptr, nullptr, cnt, m, tm, pool, s);
+        } else {
+            st = launch_dec_lay<tq3::kSoA>(bf, def, smem, packed + off * 48, norms + off, scales + off, cnt, m, tm,
+                                           pool, s);
+        }
         if (st != WQ_OK) return st;
     }
     return WQ_OK;

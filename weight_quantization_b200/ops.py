@@ -27,6 +27,8 @@ PROTOTYPES = {
     "tq3_decode": (_int, [_vp, _vp, _vp, _i64, _vp, _vp, _int, _vp]),
     "tq3_encode_aos": (_int, [_vp, _int, _i64, _vp, _vp, _vp]),
     "tq3_decode_aos": (_int, [_vp, _i64, _vp, _vp, _int, _vp]),
+    "tq3_encode_slots": (_int, [_vp, _int, _i64, _vp, _vp, _vp, _i64, _vp]),
+    "tq3_decode_paged": (_int, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _vp, _int, _vp]),
     "tq3_compressed_bytes": (_i64, [_i64]),
     "rpbh_quantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp]),
     "rpbh_dequantize_weight": (_int, [_vp, _vp, _int, _i64, _i64, _int, _vp, _vp, _vp, _int, _vp, _int, _vp]),
@@ -167,6 +169,47 @@ def tq3_decode_aos(records: torch.Tensor, sign_mask, out_dtype=torch.float32, ou
     st = lib().tq3_decode_aos(_dev(records, "records"), n_vec, m.ctypes.data, _dev(out, "out"), _DT[out.dtype],
                               _stream(records.device))
     _check("tq3_decode_aos", st)
+    return out
+
+
+def tq3_encode_slots(x: torch.Tensor, sign_mask, slots: torch.Tensor, pool: torch.Tensor):
+    """TQ3-encode the vectors of x ([..., D] fp32/bf16, D a multiple of 128, so x.numel() / 128
+    vectors) into a pool of 56-byte records [n_pool, 56]: vector v goes to record slots[v] (int64;
+    a negative slot skips the vector). Slots at or beyond n_pool are skipped and raise device fault
+    bit 6. Returns pool."""
+    if x.dtype not in _DT:
+        raise ValueError("x must be float32 or bfloat16")
+    if x.ndim == 0 or x.shape[-1] % 128 != 0 or x.shape[-1] <= 0:
+        raise ValueError("last dim must be a positive multiple of 128")
+    n_vec = x.numel() // 128
+    if slots.dtype != torch.int64 or slots.numel() != n_vec:
+        raise ValueError("slots must be int64 with one entry per vector")
+    if pool.dtype != torch.uint8 or pool.ndim != 2 or pool.shape[1] != 56:
+        raise ValueError("pool must be uint8 [n_pool, 56]")
+    m = _mask_arg(sign_mask)
+    st = lib().tq3_encode_slots(_dev(x, "x"), _DT[x.dtype], n_vec, m.ctypes.data, _dev(slots, "slots"),
+                                _dev(pool, "pool"), pool.shape[0], _stream(x.device))
+    _check("tq3_encode_slots", st)
+    return pool
+
+
+def tq3_decode_paged(pool: torch.Tensor, page_table: torch.Tensor, page_size: int, n_vec: int, sign_mask,
+                     out_dtype=torch.float32, out=None):
+    """Decode n_vec logically consecutive vectors from a pool of 56-byte records [n_pool, 56]
+    through a page table (int32): vector p is record page_table[p // page_size] * page_size +
+    p % page_size. page_size is a power of two. Returns [n_vec, 128] of out_dtype; entries outside
+    the pool decode as zeros and raise device fault bit 6."""
+    if pool.dtype != torch.uint8 or pool.ndim != 2 or pool.shape[1] != 56:
+        raise ValueError("pool must be uint8 [n_pool, 56]")
+    if page_table.dtype != torch.int32:
+        raise ValueError("page_table must be int32")
+    if out is None:
+        out = torch.empty((n_vec, 128), dtype=out_dtype, device=pool.device)
+    m = _mask_arg(sign_mask)
+    st = lib().tq3_decode_paged(_dev(pool, "pool"), pool.shape[0], _dev(page_table, "page_table"),
+                                page_table.numel(), int(page_size), int(n_vec), m.ctypes.data, _dev(out, "out"),
+                                _DT[out.dtype], _stream(pool.device))
+    _check("tq3_decode_paged", st)
     return out
 
 
