@@ -125,7 +125,7 @@ def traffic_bytes(kernel: str):
         return None
     src = {"tq3_encode": "tq3_mma.cu", "tq3_decode": "tq3_rows.cu", "tq3_encode_exact": "tq3.cu",
            "rpbh_quantize": "rpbh_fast.cu", "rpbh_rotate": "rpbh_fast.cu", "rpbh_dequantize": "rpbh_fast.cu",
-           "rpbh_linear": "rpbh_linear.cu"}.get(kernel)
+           "rpbh_linear": "rpbh_linear.cu", "tq3_attention": "tq3_attn.cu"}.get(kernel)
     if src is None:
         return None
     with open(os.path.join(ROOT, "weight_quantization_b200", "csrc", src), "rb") as f:
@@ -561,8 +561,81 @@ class RPBHLinearWorkload:
         return flops / dt, f"{done} blocks of 64 output features x 64 activation rows (dequantize + fp64 product), {dt:.1f} s"
 
 
+class TQ3AttentionWorkload:
+    """Decode-step attention over a TQ3 KV cache: 8 sequences x 8 KV heads x 32768 keys, 4 query rows
+    per KV head (32 query heads, one token), bf16 queries and outputs. K and V are 56-byte records
+    drawn with the long-context recipe (235 MB together, larger than L2)."""
+
+    metric = "TQ3 attention keys/s (key-value records attended per second)"
+    unit = "keys/s"
+
+    def __init__(self, dev, heads=64, S=32768, m=4, seed=6):
+        from weight_quantization_b200 import ops
+        self.ops = ops
+        self.name = f"tq3-attention-decode-{heads}x{S}-m{m}"
+        self.heads, self.S, self.m = heads, S, m
+        self.mask = ops.sign_mask_words(inputs.tq3_sign_bits())
+
+        def records(sd):
+            p, n, sc = (torch.from_numpy(a) for a in inputs.long_context_records(heads * S, seed=sd))
+            return torch.cat([p, n.view(torch.uint8).view(-1, 4), sc.view(torch.uint8).view(-1, 4)], 1).view(heads, S, 56)
+
+        self.kr, self.vr = records(seed).to(dev), records(seed + 1).to(dev)
+        q = torch.randn(heads, m, 128, generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16)
+        self.host_q = q
+        self.q = q.to(dev)
+        self.out = torch.empty(heads, m, 128, dtype=torch.bfloat16, device=dev)
+        self.units = heads * S
+        self.kernels = ["tq3_attention"]
+        self.bytes_per_launch = {"tq3_attention": 112 * heads * S + 2 * 2 * heads * m * 128}
+        self.l2 = "K and V records (235 MB) larger than L2, read once per launch"
+
+    rotation = 1
+
+    def _attn(self, k):
+        self.ops.tq3_attention(self.q, self.kr, self.vr, self.mask, out=self.out)
+
+    def parts(self):
+        return [("tq3_attention", 1, self._attn)]
+
+    def extras(self):
+        return []
+
+    step = KVWorkload.step
+
+    def e2e_setup(self):
+        self.pin_in = self.host_q.pin_memory()
+        self.pin_out = torch.empty(self.heads, self.m, 128, dtype=torch.bfloat16).pin_memory()
+        self.h2d = self.pin_in.numel() * 2
+        self.d2h = self.pin_out.numel() * 2
+
+    def e2e_step(self):
+        """The step's queries in from pinned memory, attention through the public call, the output
+        rows out (the cache stays resident, as in decoding)."""
+        self.q.copy_(self.pin_in, non_blocking=True)
+        self._attn(0)
+        self.pin_out.copy_(self.out, non_blocking=True)
+
+    def e2e_check(self):
+        return torch.equal(self.pin_out, self.out.cpu())
+
+    def oracle_rate(self, budget_s=10.0):
+        import oracle
+        oracle.lib()
+        bits = inputs.tq3_sign_bits()
+        q = self.host_q.float().numpy()
+        kr, vr = self.kr[:1].cpu().numpy(), self.vr[:1].cpu().numpy()
+        done, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < budget_s and done < 64:
+            oracle.tq3_attention(q[:1], kr, vr, bits, 128 ** -0.5)
+            done += 1
+        dt = time.perf_counter() - t0
+        return done * self.S / dt, f"{done} passes over head 0 ({self.S} keys, {self.m} query rows), {dt:.1f} s"
+
+
 WORKLOADS = {
     "kv": KVWorkload,
+    "tq3-attention": TQ3AttentionWorkload,
     "longctx": LongContextWorkload,
     "rpbh-llm": lambda dev: RPBHWorkload(dev),
     "rpbh-dit": lambda dev: RPBHWorkload(dev, rows=12288, d=3072, xrows=4096, bits=3, seed=4),

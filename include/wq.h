@@ -130,6 +130,28 @@ wq_status tq3_decode_paged(const uint8_t *pool, int64_t n_pool, const int32_t *p
                            int64_t page_size, int64_t n_vec, const uint32_t *sign_mask, void *out,
                            int out_dtype, void *stream);
 
+/* tq3_attention -- scaled dot-product attention over a TQ3-compressed K/V cache (page "tq3_core.py":
+ * the cache is what tq3_quantize compresses and tq3_dequantize restores; the page's commit note
+ * names the attention layer that reads it). For every head h and query row r:
+ *   out[h][r] = sum_j p_j v_j / sum_j p_j,  p_j = exp(softmax_scale * q[h][r] . k_j - max),
+ * where k_j, v_j (j = 0 .. S-1) are tq3_dequantize of the records k_records[h][j], v_records[h][j].
+ * No mask: every row attends to all S keys of its head.
+ *   q          device, heads x m x 128 elements of q_dtype. The m rows of a head share its keys and
+ *              values (grouped-query attention: m = query heads per KV head x query tokens).
+ *   m          1 .. 16.
+ *   k_records, v_records  device, heads x S x 56 bytes (the tq3_encode_aos record), 8-byte aligned.
+ *   S          1 .. 2^31 keys per head.
+ *   softmax_scale  finite; 1/sqrt(128) is the usual value.
+ *   out        device, heads x m x 128 elements of out_dtype (bf16: rounded once, to nearest even).
+ * Precision: the keys and values are never decoded; the query is rotated once into the basis the
+ * indices live in and the output rotated back once, in fp32. The result differs from attention over
+ * the decoded fp32 vectors by fp32 rounding only.
+ * Errors: WQ_ERR_SHAPE (heads < 0, m or S out of range, softmax_scale not finite), WQ_ERR_DTYPE,
+ * WQ_ERR_NULL, WQ_ERR_ALIGN (q and out to their element size). heads == 0 enqueues nothing. */
+wq_status tq3_attention(const void *q, int q_dtype, int64_t heads, int64_t m, const uint8_t *k_records,
+                        const uint8_t *v_records, int64_t S, const uint32_t *sign_mask, float softmax_scale,
+                        void *out, int out_dtype, void *stream);
+
 /* tq3_compressed_bytes -- tq3_memory_bytes' compressed size for n_vec vectors: 56 * n_vec
  * (-1 if n_vec < 0 or the product overflows). */
 int64_t tq3_compressed_bytes(int64_t n_vec);

@@ -149,6 +149,24 @@ def tq3_to_records(packed, norms, scales):
     return np.concatenate([p, n, s], axis=1)
 
 
+def tq3_attention(q, k_records, v_records, sign_bits, softmax_scale: float):
+    """Scaled dot-product attention over a TQ3 K/V cache, by definition: every key and value is
+    restored by tq3_dequantize (page "tq3_core.py", the page's own fp32 rounding), then, in fp64,
+    out[h, r] = sum_j p_j v_j / sum_j p_j with p_j = exp(softmax_scale * q[h, r] . k_j - max_j).
+    q [heads, m, 128] (fp32 values); k_records, v_records [heads, S, 56] records (tq3_to_records).
+    Returns fp64 [heads, m, 128]."""
+    q = np.asarray(q, np.float64)
+    heads, m, _ = q.shape
+    out = np.zeros((heads, m, 128), np.float64)
+    for h in range(heads):
+        k = tq3_decode(*tq3_from_records(k_records[h]), sign_bits).astype(np.float64)
+        v = tq3_decode(*tq3_from_records(v_records[h]), sign_bits).astype(np.float64)
+        logits = softmax_scale * (q[h] @ k.T)
+        p = np.exp(logits - logits.max(axis=1, keepdims=True))
+        out[h] = (p @ v) / p.sum(axis=1, keepdims=True)
+    return out
+
+
 def tq3_from_records(records):
     """The inverse of tq3_to_records: (packed [n, 48], norms [n], scales [n])."""
     r = np.ascontiguousarray(records, np.uint8).reshape(-1, 56)

@@ -1,0 +1,115 @@
+"""GPU attention over a TQ3-compressed K/V cache (tq3_attention) against the oracle, through the C ABI.
+
+The oracle decodes every key and value with the page's tq3_dequantize (page "tq3_core.py") and takes
+softmax(softmax_scale q k^T) v in fp64. The kernel never decodes: it rotates q into the indices'
+basis, scores and accumulates there in fp32, and rotates each output row back once.
+
+Tolerance, from the arithmetic (u = 2^-24, first order):
+* logits. The kernel's logit for key j is a 128-term fp32 dot product of the rotated query (seven
+  rounded butterfly stages) with the key's centroids, times norm * scale * post * softmax_scale * log2 e.
+  Bounding each rounding by u times the sum of absolute terms, and that sum by Cauchy-Schwarz, gives
+  |d logit_j| <= (128 + 7 sqrt(128) + 10) u * softmax_scale |q| |k_j| < 2^-16 softmax_scale |q| max_j |k_j|
+  =: L (the last 10 u cover the page's own rounding of k_j, the coefficient and the max subtraction).
+* weights. Logits off by at most L change every normalised weight by a factor within e^(+-2L), so
+  the output moves by at most (e^(4L) - 1) max_j |v_j|_inf <= 4.4 L max_j |v_j|_inf; exp2f adds
+  2^-21 max_j |v_j|_inf.
+* values. Each rotated accumulator sums n = ceil(S / splits) + 8 weighted centroids in fp32 (the
+  running sum over this CTA's keys, then the cluster merge), and the inverse transform adds seven
+  stages; bounded as above this is (n + 40) u max_j |v_j|_2 on every output element.
+* bf16 output: one rounding, 2^-8 |out| allowed.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from weight_quantization_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+U = 2.0 ** -24
+
+
+@pytest.fixture(scope="module")
+def wq():
+    from weight_quantization_b200 import build, ops
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return ops
+
+
+def _cache(oracle, heads, S, seed):
+    """Records of a K and a V cache: Gaussian vectors with a per-token offset, as in the KV recipe."""
+    bits = inputs.tq3_sign_bits()
+    recs, dec = [], []
+    for i in range(2):
+        x = inputs.gaussian((heads * S, 128), seed=seed + i).astype(np.float32)
+        x += 2.0 * inputs.gaussian((heads * S, 1), seed=seed + 10 + i).astype(np.float32)
+        r = oracle.tq3_to_records(*oracle.tq3_encode(x, bits))
+        recs.append(r.reshape(heads, S, 56))
+        dec.append(oracle.tq3_decode(*oracle.tq3_from_records(r), bits).astype(np.float64).reshape(heads, S, 128))
+    return bits, recs, dec
+
+
+def _check(wq, oracle, heads, m, S, q_bf16, out_bf16, scale, seed):
+    bits, (kr, vr), (k, v) = _cache(oracle, heads, S, seed)
+    qf = (inputs.gaussian((heads, m, 128), seed=seed + 5) * 1.5).astype(np.float32)
+    if q_bf16:
+        qb = oracle.f32_array_to_bf16(qf)
+        qf = oracle.bf16_array_to_f32(qb).reshape(heads, m, 128)
+        q_dev = torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16).cuda()
+    else:
+        q_dev = torch.from_numpy(qf).cuda()
+    out = wq.tq3_attention(q_dev, torch.from_numpy(kr).cuda(), torch.from_numpy(vr).cuda(), wq.sign_mask_words(bits),
+                           softmax_scale=scale, out_dtype=torch.bfloat16 if out_bf16 else torch.float32)
+    torch.cuda.synchronize()
+    if out_bf16:
+        got = oracle.bf16_array_to_f32(out.cpu().view(torch.int16).numpy().view(np.uint16)).astype(np.float64)
+    else:
+        got = out.cpu().numpy().astype(np.float64)
+    ref = oracle.tq3_attention(qf, kr, vr, bits, scale)
+    splits = min(8, -(-S // 128))
+    n = -(-S // splits) + 8
+    vinf = np.abs(v).max(axis=(1, 2))                   # per head
+    v2 = np.linalg.norm(v, axis=2).max(axis=1)
+    k2 = np.linalg.norm(k, axis=2).max(axis=1)
+    L = 2.0 ** -16 * scale * np.linalg.norm(qf.astype(np.float64), axis=2) * k2[:, None]   # [heads, m]
+    tol = (4.4 * L + 2.0 ** -21)[:, :, None] * vinf[:, None, None] + ((n + 40) * U * v2)[:, None, None]
+    if out_bf16:
+        tol = tol + 2.0 ** -8 * np.abs(ref)
+    err = np.abs(got - ref)
+    worst = float((err / tol).max())
+    assert worst <= 1.0, f"worst error {worst:.3f} of the tolerance (max abs err {err.max():.3g})"
+    return worst
+
+
+@pytest.mark.parametrize("heads,m,S", [(1, 1, 1), (3, 4, 127), (2, 8, 1000), (5, 16, 4097), (2, 3, 128 * 8 * 3 + 5),
+                                       (4, 2, 129)])
+@pytest.mark.parametrize("q_bf16", [True, False])
+def test_attention_matches_oracle(wq, oracle, heads, m, S, q_bf16):
+    _check(wq, oracle, heads, m, S, q_bf16, False, 128 ** -0.5, seed=heads * 1000 + m * 10 + S)
+
+
+@pytest.mark.parametrize("m", [1, 5, 8])
+def test_attention_bf16_out_and_sharp_softmax(wq, oracle, m):
+    _check(wq, oracle, 3, m, 2000, True, True, 0.5, seed=7 + m)
+
+
+def test_attention_long_context(wq, oracle):
+    """32768 keys per head: the full cluster split, long per-CTA accumulations."""
+    _check(wq, oracle, 2, 8, 32768, True, False, 128 ** -0.5, seed=31)
+
+
+def test_attention_argument_errors(wq):
+    from weight_quantization_b200.ops import WQError
+    mask = wq.sign_mask_words(inputs.tq3_sign_bits())
+    rec = torch.zeros(2, 16, 56, dtype=torch.uint8, device="cuda")
+    with pytest.raises(WQError):  # more than 16 rows per head
+        wq.tq3_attention(torch.zeros(2, 17, 128, device="cuda"), rec, rec, mask)
+    with pytest.raises(WQError):  # no keys
+        empty = torch.zeros(2, 0, 56, dtype=torch.uint8, device="cuda")
+        wq.tq3_attention(torch.zeros(2, 1, 128, device="cuda"), empty, empty, mask)
+    with pytest.raises(WQError):
+        wq.tq3_attention(torch.zeros(2, 1, 128, device="cuda"), rec, rec, mask, softmax_scale=math.inf)
+    assert wq.tq3_attention(torch.zeros(0, 1, 128, device="cuda"), rec[:0], rec[:0], mask).shape == (0, 1, 128)

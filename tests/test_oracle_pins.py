@@ -518,3 +518,49 @@ def test_rpbh_rotate_bf16_matches_dense(oracle):
     got = oracle.bf16_array_to_f32(out).astype(np.float64)
     # one bf16 rounding of a value that is itself within 1e-6 of the float64 result
     assert np.all(np.abs(got - ref) <= np.abs(ref) * 2 ** -8 + 1e-6)
+
+
+def _attn_cache(oracle, heads, S, seed, same_keys=False):
+    bits = inputs.tq3_sign_bits()
+    x = inputs.gaussian((2, heads, S, 128), seed=seed).astype(np.float32)
+    if same_keys:
+        x[:, :, :, :] = x[:, :, :1, :]
+    recs = [oracle.tq3_to_records(*oracle.tq3_encode(x[i].reshape(-1, 128), bits)).reshape(heads, S, 56)
+            for i in range(2)]
+    dec = [oracle.tq3_decode(*oracle.tq3_from_records(r.reshape(-1, 56)), bits).reshape(heads, S, 128)
+           .astype(np.float64) for r in recs]
+    return bits, recs[0], recs[1], dec[0], dec[1]
+
+
+def test_tq3_attention_closed_forms(oracle):
+    """Attention over the decoded cache: one key returns its value; identical keys return their
+    value whatever the query; a zero query averages the values; permuting the keys together with
+    their values changes nothing."""
+    bits, kr, vr, k, v = _attn_cache(oracle, 2, 1, seed=80)
+    q = inputs.gaussian((2, 3, 128), seed=81).astype(np.float32)
+    assert np.allclose(oracle.tq3_attention(q, kr, vr, bits, 0.088), np.repeat(v, 3, axis=1), rtol=0, atol=1e-12)
+
+    bits, kr, vr, k, v = _attn_cache(oracle, 1, 9, seed=82, same_keys=True)
+    out = oracle.tq3_attention(q[:1], kr, vr, bits, 0.5)
+    assert np.allclose(out, np.repeat(v[:, :1], 3, axis=1), rtol=0, atol=1e-12)
+
+    bits, kr, vr, k, v = _attn_cache(oracle, 2, 17, seed=83)
+    out = oracle.tq3_attention(np.zeros((2, 2, 128), np.float32), kr, vr, bits, 0.3)
+    assert np.allclose(out, np.repeat(v.mean(axis=1, keepdims=True), 2, axis=1), rtol=0, atol=1e-12)
+
+    q = inputs.gaussian((2, 4, 128), seed=84).astype(np.float32)
+    perm = np.random.default_rng(0).permutation(17)
+    a = oracle.tq3_attention(q, kr, vr, bits, 0.1)
+    b = oracle.tq3_attention(q, kr[:, perm], vr[:, perm], bits, 0.1)
+    assert np.allclose(a, b, rtol=0, atol=1e-12)
+
+
+def test_tq3_attention_hard_max_picks_the_value_of_the_best_key(oracle):
+    """With a large softmax scale the weights collapse onto the key with the largest q . k: the
+    output is that key's value (not its key, and not the value of the smallest q . k)."""
+    bits, kr, vr, k, v = _attn_cache(oracle, 1, 12, seed=85)
+    q = inputs.gaussian((1, 2, 128), seed=86).astype(np.float32)
+    out = oracle.tq3_attention(q, kr, vr, bits, 1e4)
+    for r in range(2):
+        best = int(np.argmax(k[0] @ q[0, r].astype(np.float64)))
+        assert np.allclose(out[0, r], v[0, best], rtol=0, atol=1e-9)

@@ -29,6 +29,7 @@ PROTOTYPES = {
     "tq3_decode_aos": (_int, [_vp, _i64, _vp, _vp, _int, _vp]),
     "tq3_encode_slots": (_int, [_vp, _int, _i64, _vp, _vp, _vp, _i64, _vp]),
     "tq3_decode_paged": (_int, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _vp, _int, _vp]),
+    "tq3_attention": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _vp, C.c_float, _vp, _int, _vp]),
     "tq3_compressed_bytes": (_i64, [_i64]),
     "rpbh_quantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp]),
     "rpbh_dequantize_weight": (_int, [_vp, _vp, _int, _i64, _i64, _int, _vp, _vp, _vp, _int, _vp, _int, _vp]),
@@ -210,6 +211,29 @@ def tq3_decode_paged(pool: torch.Tensor, page_table: torch.Tensor, page_size: in
                                 page_table.numel(), int(page_size), int(n_vec), m.ctypes.data, _dev(out, "out"),
                                 _DT[out.dtype], _stream(pool.device))
     _check("tq3_decode_paged", st)
+    return out
+
+
+def tq3_attention(q: torch.Tensor, k_records: torch.Tensor, v_records: torch.Tensor, sign_mask,
+                  softmax_scale: float = 128 ** -0.5, out_dtype=None, out=None):
+    """Attention of q [heads, m, 128] (fp32/bf16; the m rows of a head share its keys and values,
+    e.g. the query heads of one KV head) over TQ3 records k_records, v_records [heads, S, 56]:
+    softmax(softmax_scale * q k^T) v with k, v the decoded records. Returns [heads, m, 128]."""
+    if q.dtype not in _DT or q.ndim != 3 or q.shape[2] != 128:
+        raise ValueError("q must be [heads, m, 128] float32 or bfloat16")
+    heads, m = q.shape[0], q.shape[1]
+    for name, t in (("k_records", k_records), ("v_records", v_records)):
+        if t.dtype != torch.uint8 or t.ndim != 3 or t.shape[0] != heads or t.shape[2] != 56:
+            raise ValueError(f"{name} must be uint8 [heads, S, 56]")
+    if k_records.shape != v_records.shape:
+        raise ValueError("k_records and v_records must have the same shape")
+    if out is None:
+        out = torch.empty((heads, m, 128), dtype=out_dtype or q.dtype, device=q.device)
+    msk = _mask_arg(sign_mask)
+    st = lib().tq3_attention(_dev(q, "q"), _DT[q.dtype], heads, m, _dev(k_records, "k_records"),
+                             _dev(v_records, "v_records"), k_records.shape[1], msk.ctypes.data,
+                             float(softmax_scale), _dev(out, "out"), _DT[out.dtype], _stream(q.device))
+    _check("tq3_attention", st)
     return out
 
 
