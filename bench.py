@@ -679,7 +679,10 @@ def max_over_ranks(x: float, world: int) -> float:
 def run_ours(args):
     world, rank, local = dist_setup(args)
     dev = torch.device("cuda", local)
-    wl = WORKLOADS[args.workload](dev)
+    if args.workload == "tq3-attention":
+        wl = TQ3AttentionWorkload(dev, m=args.attn_rows)
+    else:
+        wl = WORKLOADS[args.workload](dev)
     parts = wl.parts()
     # eager warm-up (loads the library, sets kernel attributes). The timed steps are then replayed
     # from CUDA graphs that hold up to CHUNK consecutive steps each (host launch overhead and
@@ -878,6 +881,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-chunk", type=int, default=2048)
+    ap.add_argument("--attn-rows", type=int, default=4,
+                    help="query rows per KV head for --workload tq3-attention (1..16)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
