@@ -121,3 +121,56 @@ def test_sign_mask_layout(wq):
     m = wq.sign_mask_words(bits)
     assert np.array_equal(m, inputs.tq3_sign_mask_words(bits))
     assert [hex(v) for v in m] == ["0x3fd74222", "0x1ab7c17", "0xff4abaf6", "0x656b5fe7"]
+
+
+def test_record_pool_and_attention_argument_validation(wq):
+    """tq3_encode_aos / tq3_decode_aos / tq3_encode_slots / tq3_decode_paged / tq3_attention reject bad
+    arguments with their documented codes before any device work (fake device addresses)."""
+    L = wq.lib()
+    m = np.zeros(4, np.uint32)
+    mp = m.ctypes.data
+    A = 0x10000
+    assert L.tq3_encode_aos(A, 1, 0, mp, A, None) == WQ_OK
+    assert L.tq3_encode_aos(A, 1, -1, mp, A, None) == WQ_ERR_SHAPE
+    assert L.tq3_encode_aos(A, 1, 4, mp, A + 4, None) == WQ_ERR_ALIGN      # records need 8 bytes
+    assert L.tq3_decode_aos(A, 4, mp, A + 8, 1, None) == WQ_ERR_ALIGN      # out needs 16 bytes
+    assert L.tq3_decode_aos(None, 4, mp, A, 1, None) == WQ_ERR_NULL
+
+    slots = lambda x=A, dt=1, n=4, msk=mp, sl=A, pool=A, n_pool=8: L.tq3_encode_slots(x, dt, n, msk, sl, pool, n_pool, None)
+    assert slots(n=0) == WQ_OK
+    assert slots(n=-1) == WQ_ERR_SHAPE
+    assert slots(n_pool=-1) == WQ_ERR_SHAPE
+    assert slots(dt=9) == WQ_ERR_DTYPE
+    assert slots(sl=None) == WQ_ERR_NULL
+    assert slots(pool=A + 4) == WQ_ERR_ALIGN
+    assert slots(sl=A + 4) == WQ_ERR_ALIGN
+    assert slots(x=A + 8) == WQ_ERR_ALIGN
+
+    paged = lambda pool=A, n_pool=64, tab=A, n_pages=4, ps=16, n=64, out=A, dt=1: \
+        L.tq3_decode_paged(pool, n_pool, tab, n_pages, ps, n, mp, out, dt, None)
+    assert paged(n=0) == WQ_OK
+    for ps in (0, 12, 3, 1 << 31):
+        assert paged(ps=ps) == WQ_ERR_SHAPE                                # a power of two, 1 .. 2^30
+    assert paged(n=65) == WQ_ERR_SHAPE                                     # more than the table covers
+    assert paged(n_pages=-1) == WQ_ERR_SHAPE
+    assert paged(dt=2) == WQ_ERR_DTYPE
+    assert paged(tab=None) == WQ_ERR_NULL
+    assert paged(tab=A + 2) == WQ_ERR_ALIGN
+    assert paged(pool=A + 4) == WQ_ERR_ALIGN
+    assert paged(out=A + 8) == WQ_ERR_ALIGN
+
+    attn = lambda q=A, qdt=1, heads=2, rows=4, k=A, v=A, S=100, scale=0.088, out=A, odt=1: \
+        L.tq3_attention(q, qdt, heads, rows, k, v, S, mp, scale, out, odt, None)
+    assert attn(heads=0) == WQ_OK
+    for rows in (0, 17):
+        assert attn(rows=rows) == WQ_ERR_SHAPE
+    for S in (0, (1 << 31) + 1):
+        assert attn(S=S) == WQ_ERR_SHAPE
+    assert attn(heads=-1) == WQ_ERR_SHAPE
+    assert attn(scale=float("inf")) == WQ_ERR_SHAPE
+    assert attn(scale=float("nan")) == WQ_ERR_SHAPE
+    assert attn(qdt=5) == WQ_ERR_DTYPE
+    assert attn(v=None) == WQ_ERR_NULL
+    assert attn(k=A + 4) == WQ_ERR_ALIGN
+    assert attn(q=A + 1) == WQ_ERR_ALIGN                                   # bf16 needs 2 bytes
+    assert attn(out=A + 2, odt=0) == WQ_ERR_ALIGN                          # fp32 needs 4 bytes
