@@ -20,8 +20,8 @@
 // accumulators per query row (online softmax), and the cluster combines its CTAs' partial results
 // through distributed shared memory, so nothing is written to global memory but the output. Within
 // a CTA, thread t scores key t of the tile (its indices are unpacked once and serve every query
-// row); for the values, each lane owns four rotated coordinates and each warp a quarter or an
-// eighth of the tile's keys, the warps' sums being added once at the end.
+// row); for the values, each lane owns four rotated coordinates and each warp a quarter of the
+// tile's keys, the warps' sums being added once at the end.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <math.h>
