@@ -7,6 +7,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 from conftest import ROOT
 from weight_quantization_b200 import inputs
@@ -174,3 +175,32 @@ def test_record_pool_and_attention_argument_validation(wq):
     assert attn(k=A + 4) == WQ_ERR_ALIGN
     assert attn(q=A + 1) == WQ_ERR_ALIGN                                   # bf16 needs 2 bytes
     assert attn(out=A + 2, odt=0) == WQ_ERR_ALIGN                          # fp32 needs 4 bytes
+
+
+def test_bindings_reject_buffers_smaller_than_the_call(wq):
+    """The C ABI takes plain pointers, so the Python binding checks every caller-supplied buffer's
+    size first: a short one raises ValueError before any device work (CPU tensors suffice)."""
+    mask = np.zeros(4, np.uint32)
+    p, n, s = torch.zeros(4, 48, dtype=torch.uint8), torch.zeros(4), torch.zeros(4)
+    with pytest.raises(ValueError, match="out holds"):
+        wq.tq3_decode(p, n, s, mask, out=torch.empty(4 * 128 - 1))
+    with pytest.raises(ValueError, match="packed holds"):
+        wq.tq3_encode(torch.zeros(4, 128), mask, packed=torch.empty(4 * 48 - 1, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="records holds"):
+        wq.tq3_encode_aos(torch.zeros(4, 128), mask, records=torch.empty(4 * 56 - 8, dtype=torch.uint8))
+    with pytest.raises(ValueError, match="out holds"):
+        wq.tq3_decode_aos(torch.zeros(4, 56, dtype=torch.uint8), mask, out=torch.empty(3, 128))
+    with pytest.raises(ValueError, match="out holds"):
+        wq.tq3_decode_paged(torch.zeros(64, 56, dtype=torch.uint8), torch.zeros(4, dtype=torch.int32), 16, 64, mask,
+                            out=torch.empty(63, 128))
+    rec = torch.zeros(2, 10, 56, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="out holds"):
+        wq.tq3_attention(torch.zeros(2, 4, 128), rec, rec, mask, out=torch.empty(2, 3, 128))
+    perm, signs = torch.zeros(63, dtype=torch.int32), torch.ones(64, dtype=torch.int8)
+    with pytest.raises(ValueError, match="perm holds"):
+        wq.rpbh_rotate_activations(torch.zeros(4, 64), perm, signs)
+    cb = np.linspace(-1, 1, 8, dtype=np.float32)
+    with pytest.raises(ValueError, match="packed holds"):
+        wq.rpbh_dequantize_weight(torch.zeros(95, dtype=torch.uint8), torch.zeros(4), 4, 64, 3, cb)
+    with pytest.raises(ValueError, match="row_norms holds"):
+        wq.rpbh_linear(torch.zeros(96, dtype=torch.uint8), torch.zeros(3), 4, 64, 3, cb, torch.zeros(2, 64))

@@ -81,6 +81,13 @@ def _dev(t: torch.Tensor, name: str) -> int:
     return t.data_ptr()
 
 
+def _fits(t, n: int, name: str):
+    """The library takes plain pointers: a buffer smaller than what the call reads or writes is
+    rejected here, before any device work."""
+    if t is not None and t.numel() < n:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call needs {n}")
+
+
 def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
@@ -119,6 +126,9 @@ def tq3_encode(x: torch.Tensor, sign_mask, packed=None, norms=None, scales=None,
         norms = torch.empty(lead, dtype=torch.float32, device=x.device)
     if scales is None:
         scales = torch.empty(lead, dtype=torch.float32, device=x.device)
+    _fits(packed, 48 * n_vec, "packed")
+    _fits(norms, n_vec, "norms")
+    _fits(scales, n_vec, "scales")
     m = _mask_arg(sign_mask)
     name = "tq3_encode_exact" if exact else "tq3_encode"
     st = getattr(lib(), name)(_dev(x, "x"), _DT[x.dtype], n_vec, m.ctypes.data, _dev(packed, "packed"),
@@ -135,6 +145,7 @@ def tq3_decode(packed: torch.Tensor, norms: torch.Tensor, scales: torch.Tensor, 
     n_vec = norms.numel()
     if out is None:
         out = torch.empty(tuple(norms.shape) + (128,), dtype=out_dtype, device=packed.device)
+    _fits(out, 128 * n_vec, "out")
     m = _mask_arg(sign_mask)
     st = lib().tq3_decode(_dev(packed, "packed"), _dev(norms, "norms"), _dev(scales, "scales"), n_vec,
                           m.ctypes.data, _dev(out, "out"), _DT[out.dtype], _stream(packed.device))
@@ -152,6 +163,7 @@ def tq3_encode_aos(x: torch.Tensor, sign_mask, records=None):
     lead = tuple(x.shape[:-1]) + (x.shape[-1] // 128,)
     if records is None:
         records = torch.empty(lead + (56,), dtype=torch.uint8, device=x.device)
+    _fits(records, 56 * (x.numel() // 128), "records")
     m = _mask_arg(sign_mask)
     st = lib().tq3_encode_aos(_dev(x, "x"), _DT[x.dtype], x.numel() // 128, m.ctypes.data, _dev(records, "records"),
                               _stream(x.device))
@@ -166,6 +178,7 @@ def tq3_decode_aos(records: torch.Tensor, sign_mask, out_dtype=torch.float32, ou
     n_vec = records.numel() // 56
     if out is None:
         out = torch.empty(tuple(records.shape[:-1]) + (128,), dtype=out_dtype, device=records.device)
+    _fits(out, 128 * n_vec, "out")
     m = _mask_arg(sign_mask)
     st = lib().tq3_decode_aos(_dev(records, "records"), n_vec, m.ctypes.data, _dev(out, "out"), _DT[out.dtype],
                               _stream(records.device))
@@ -206,6 +219,7 @@ def tq3_decode_paged(pool: torch.Tensor, page_table: torch.Tensor, page_size: in
         raise ValueError("page_table must be int32")
     if out is None:
         out = torch.empty((n_vec, 128), dtype=out_dtype, device=pool.device)
+    _fits(out, 128 * n_vec, "out")
     m = _mask_arg(sign_mask)
     st = lib().tq3_decode_paged(_dev(pool, "pool"), pool.shape[0], _dev(page_table, "page_table"),
                                 page_table.numel(), int(page_size), int(n_vec), m.ctypes.data, _dev(out, "out"),
@@ -229,6 +243,7 @@ def tq3_attention(q: torch.Tensor, k_records: torch.Tensor, v_records: torch.Ten
         raise ValueError("k_records and v_records must have the same shape")
     if out is None:
         out = torch.empty((heads, m, 128), dtype=out_dtype or q.dtype, device=q.device)
+    _fits(out, heads * m * 128, "out")
     msk = _mask_arg(sign_mask)
     st = lib().tq3_attention(_dev(q, "q"), _DT[q.dtype], heads, m, _dev(k_records, "k_records"),
                              _dev(v_records, "v_records"), k_records.shape[1], msk.ctypes.data,
@@ -264,6 +279,10 @@ def rpbh_quantize_weight(W: torch.Tensor, perm: torch.Tensor, signs: torch.Tenso
         packed = torch.empty(max(rpbh_packed_bytes(rows, d, bits), 0), dtype=torch.uint8, device=W.device)
     if row_norms is None:
         row_norms = torch.empty(rows, dtype=W.dtype, device=W.device)
+    _fits(packed, rpbh_packed_bytes(rows, d, bits), "packed")
+    _fits(row_norms, rows, "row_norms")
+    _fits(perm, d, "perm")
+    _fits(signs, d, "signs")
     st = lib().rpbh_quantize_weight(_dev(W, "W"), _DT.get(W.dtype, -1), rows, d, _dev(perm, "perm"),
                                     _dev(signs, "signs"), bits, cb.ctypes.data, _dev(packed, "packed"),
                                     _dev(row_norms, "row_norms"), _stream(W.device))
@@ -277,6 +296,11 @@ def rpbh_dequantize_weight(packed: torch.Tensor, row_norms: torch.Tensor, rows: 
     cb = _codebook_arg(codebook, bits)
     if out is None:
         out = torch.empty(rows, d, dtype=out_dtype, device=packed.device)
+    _fits(packed, rpbh_packed_bytes(rows, d, bits), "packed")
+    _fits(row_norms, rows, "row_norms")
+    _fits(out, rows * d, "out")
+    _fits(perm, d, "perm")
+    _fits(signs, d, "signs")
     pp = _dev(perm, "perm") if perm is not None else None
     sp = _dev(signs, "signs") if signs is not None else None
     st = lib().rpbh_dequantize_weight(_dev(packed, "packed"), _dev(row_norms, "row_norms"),
@@ -292,6 +316,9 @@ def rpbh_rotate_activations(x: torch.Tensor, perm: torch.Tensor, signs: torch.Te
     rows, d = x.shape
     if out is None:
         out = torch.empty_like(x)
+    _fits(out, rows * d, "out")
+    _fits(perm, d, "perm")
+    _fits(signs, d, "signs")
     st = lib().rpbh_rotate_activations(_dev(x, "x"), _DT.get(x.dtype, -1), rows, d, _dev(perm, "perm"),
                                        _dev(signs, "signs"), _dev(out, "out"), _stream(x.device))
     _check("rpbh_rotate_activations", st)
@@ -305,6 +332,11 @@ def rpbh_linear(packed: torch.Tensor, row_norms: torch.Tensor, out_features: int
     m = x_rot.shape[0]
     if out is None:
         out = torch.empty(m, out_features, dtype=torch.bfloat16, device=x_rot.device)
+    _fits(packed, rpbh_packed_bytes(out_features, d, bits), "packed")
+    _fits(row_norms, out_features, "row_norms")
+    _fits(x_rot, m * d, "x_rot")
+    _fits(bias, out_features, "bias")
+    _fits(out, m * out_features, "y")
     bp = _dev(bias, "bias") if bias is not None else None
     st = lib().rpbh_linear(_dev(packed, "packed"), _dev(row_norms, "row_norms"), _DT.get(row_norms.dtype, -1),
                            out_features, d, bits, cb.ctypes.data, _dev(x_rot, "x_rot"), m, bp, _dev(out, "y"),
