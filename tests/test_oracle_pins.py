@@ -564,3 +564,28 @@ def test_tq3_attention_hard_max_picks_the_value_of_the_best_key(oracle):
     for r in range(2):
         best = int(np.argmax(k[0] @ q[0, r].astype(np.float64)))
         assert np.allclose(out[0, r], v[0, best], rtol=0, atol=1e-9)
+
+
+def test_tq3_dot_products_in_the_indices_basis(oracle):
+    """The decoded vector is k = s . H(c[idx] scale) post norm with H the symmetric Sylvester matrix,
+    so q . k = norm scale post (H (s . q)) . c[idx] and sum_j w_j k_j = s . H(sum_j w_j norm_j scale_j
+    c[idx_j]) post: attention can score and sum without decoding. Checked in fp64 against the
+    oracle's decoded fp32 vectors (agreement to fp32 rounding)."""
+    bits = inputs.tq3_sign_bits()
+    x = inputs.gaussian((40, 128), seed=88).astype(np.float32)
+    p, n, sc = oracle.tq3_encode(x, bits)
+    k = oracle.tq3_decode(p, n, sc, bits).astype(np.float64)
+    c, _ = oracle.tq3_tables()
+    cv = c[oracle.tq3_unpack(p)].astype(np.float64)                       # [40, 128] centroids
+    s = oracle.tq3_signs(bits).astype(np.float64)
+    H = oracle.hadamard_dense(128).astype(np.float64)
+    post = float(np.float32(1.0 / np.sqrt(128.0)))
+    coef = n.astype(np.float64) * sc.astype(np.float64) * post
+    q = inputs.gaussian((3, 128), seed=89).astype(np.float64)
+    direct = q @ k.T
+    rotated = ((H @ (s * q).T).T @ cv.T) * coef[None, :]
+    assert np.abs(direct - rotated).max() <= 1e-5 * np.abs(q).sum(axis=1).max() * np.abs(k).max()
+    w = inputs.gaussian((40,), seed=90).astype(np.float64)
+    direct_v = w @ k
+    rotated_v = s * (H @ ((w * coef) @ cv))
+    assert np.abs(direct_v - rotated_v).max() <= 1e-5 * np.abs(w).sum() * np.abs(k).max()
