@@ -51,7 +51,7 @@ def _quantize_and_check(wq, oracle, w, is_bf16, d, bits):
 
 
 @pytest.mark.parametrize("d,rows", [(32, 5), (96, 37), (192, 11), (256, 3), (1024, 9), (3072, 17), (640, 1),
-                                    (4096, 3), (12288, 2), (6400, 7), (9472, 5)])
+                                    (4096, 3), (12288, 2), (6400, 7), (9472, 5), (1536, 3), (6144, 2)])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 @pytest.mark.parametrize("is_bf16", [False, True])
 def test_quantize_small(wq, oracle, d, rows, bits, is_bf16):
@@ -90,7 +90,7 @@ def test_quantize_dit_weights_full_size(wq, oracle, rows):
 
 
 @pytest.mark.parametrize("d,rows,bits", [(96, 7, 2), (192, 3, 3), (1024, 5, 3), (3072, 33, 4), (11008, 4, 3),
-                                         (4096, 2, 2)])
+                                         (4096, 2, 2), (1536, 3, 3), (6144, 2, 4)])
 @pytest.mark.parametrize("norm_bf16", [False, True])
 @pytest.mark.parametrize("out_bf16", [False, True])
 @pytest.mark.parametrize("unrotate", [False, True])
@@ -139,7 +139,7 @@ def test_quantize_then_dequantize_llm_roundtrip(wq, oracle):
 
 
 @pytest.mark.parametrize("rows,d", [(2048, 11008), (4096, 3072), (3, 96), (1, 32), (5, 192), (3, 4096),
-                                    (7, 640), (9, 2880), (5, 6400)])
+                                    (7, 640), (9, 2880), (5, 6400), (3, 1536), (2, 6144)])
 def test_rotate_activations(wq, oracle, rows, d):
     perm, signs, perm_d, signs_d = _params(d)
     h = d & -d
