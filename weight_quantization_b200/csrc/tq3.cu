@@ -396,7 +396,7 @@ extern "C" wq_status tq3_decode_paged(const uint8_t *pool, int64_t n_pool, const
     if (n_vec == 0) return WQ_OK;
     if (!pool || !page_table || !sign_mask || !out) return WQ_ERR_NULL;
     if (n_vec > ((int64_t)1 << 40) || n_pool > ((int64_t)1 << 40) || n_pages > ((int64_t)1 << 40)) return WQ_ERR_SHAPE;
-    if (n_vec > n_pages * page_size) return WQ_ERR_SHAPE;  // the table must cover every vector read
+    if ((n_vec + page_size - 1) / page_size > n_pages) return WQ_ERR_SHAPE;  // the table must cover every vector read
     if (!aligned(pool, 8) || !aligned(page_table, 4) || !aligned(out, 16)) return WQ_ERR_ALIGN;
     tq3::SignMask m;
     for (int i = 0; i < 4; ++i) m.w[i] = sign_mask[i];
