@@ -5,7 +5,7 @@
  * Sources. Every entry point restates an operation of one of two pages:
  *   "tq3_core.py" (ComfyUI-TurboQuant): module docstring (format and algorithm), tq3_quantize,
  *       tq3_dequantize, _fwht_inplace, _quantize_to_indices, _pack_3bit, _unpack_3bit,
- *       tq3_memory_bytes.
+ *       tq3_memory_bytes, and the page's commit note (the attention layer that reads the cache).
  *   "orbit_quant.py" (OrbitQuant weight-only backend): gaussian_lloyd_max, hadamard_block_size,
  *       rpbh_forward, rpbh_inverse, _fwht, pack_codes, unpack_codes, _quantize_rows,
  *       OrbitQuantizer.quantize_, _dequantize_rotated, dequantize, forward.
@@ -21,8 +21,9 @@
  *   - An empty problem (n_vec == 0, rows == 0) returns WQ_OK and enqueues nothing; its pointers
  *     may then be NULL.
  *   - Element types: WQ_F32 = IEEE binary32, WQ_BF16 = bfloat16 (raw 16-bit patterns).
- *   - All arithmetic is fp32 in the order the pages give, except the two L2 norms, whose
- *     squares are summed in fp64 and rounded once to fp32 after the square root.
+ *   - Unless an entry point states otherwise (tq3_encode, rpbh_linear, tq3_attention reorder the
+ *     arithmetic and say how), all arithmetic is fp32 in the order the pages give, except the two
+ *     L2 norms, whose squares are summed in fp64 and rounded once to fp32 after the square root.
  */
 #ifndef WQ_H
 #define WQ_H
@@ -55,8 +56,9 @@ typedef enum { WQ_F32 = 0, WQ_BF16 = 1 } wq_dtype;
 /* ============================================================================================
  * TQ3 ("tq3_core.py")
  * A TQ3 record encodes one 128-element vector as 48 bytes of 3-bit indices plus an fp32 norm
- * and an fp32 scale (56 bytes, 3.5 bits per value; module docstring). Records are stored as
- * three arrays: packed[n_vec][48], norms[n_vec], scales[n_vec] (the dict tq3_quantize returns).
+ * and an fp32 scale (56 bytes, 3.5 bits per value; module docstring). tq3_encode / tq3_decode
+ * store records as three arrays: packed[n_vec][48], norms[n_vec], scales[n_vec] (the dict
+ * tq3_quantize returns); the _aos, pool and attention calls use one 56-byte record per vector.
  * A [..., D] tensor with D a multiple of 128 is n_vec = numel / 128 consecutive vectors.
  * ============================================================================================ */
 
