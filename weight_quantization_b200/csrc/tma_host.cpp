@@ -44,15 +44,27 @@ bool make_tmap_2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, ui
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A launch may use 48 KiB of shared memory in total (static + dynamic) without opting in. The
+// kernel's static shared memory is read from its attributes, so a dynamic size just under 48 KiB
+// on a kernel that also declares __shared__ arrays still gets the opt-in it needs. The attribute
+// is raised once per (kernel, device) to the largest dynamic size asked for so far.
 bool ensure_dynamic_smem(const void *kernel, size_t smem) {
-    if (smem <= 48 * 1024) return true;
+    if (smem == 0) return true;
     static std::mutex mu;
-    static std::map<std::pair<const void *, int>, size_t> set_to;
+    static std::map<std::pair<const void *, int>, std::pair<size_t, size_t>> state;  // (static bytes, set to)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     std::lock_guard<std::mutex> lock(mu);
-    size_t &cur = set_to[std::make_pair(kernel, dev)];
-    if (smem <= cur) return true;
+    const auto key = std::make_pair(kernel, dev);
+    auto it = state.find(key);
+    if (it == state.end()) {
+        cudaFuncAttributes attr;
+        if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return false;
+        it = state.emplace(key, std::make_pair((size_t)attr.sharedSizeBytes, (size_t)0)).first;
+    }
+    const size_t static_bytes = it->second.first;
+    size_t &cur = it->second.second;
+    if (smem <= cur || static_bytes + smem <= 48 * 1024) return true;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return false;
     cur = smem;
