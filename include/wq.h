@@ -143,7 +143,10 @@ wq_status tq3_decode_paged(const uint8_t *pool, int64_t n_pool, const int32_t *p
  *   m          1 .. 16.
  *   k_records, v_records  device, heads x S x 56 bytes (the tq3_encode_aos record), 8-byte aligned.
  *   S          1 .. 2^31 keys per head.
- *   softmax_scale  finite; 1/sqrt(128) is the usual value.
+ *   softmax_scale  finite; 1/sqrt(128) is the usual value. (Any finite fp32 scale keeps the
+ *              kernel's coefficient scale * 2^-3.5 * log2(e) finite, as that factor is below 1.)
+ *              The logits softmax_scale * q . k_j themselves must be finite in fp32: a logit that
+ *              overflows makes the head's output undefined, as NaN or Inf inputs do.
  *   out        device, heads x m x 128 elements of out_dtype (bf16: rounded once, to nearest even).
  * Precision: the keys and values are never decoded; the query is rotated once into the basis the
  * indices live in and the output rotated back once, in fp32. The result differs from attention over

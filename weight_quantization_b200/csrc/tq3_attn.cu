@@ -378,6 +378,7 @@ extern "C" wq_status tq3_attention(const void *q, int q_dtype, int64_t heads, in
     float post;
     memcpy(&post, &post_bits, sizeof post);
     const float coef = (float)((double)post * (double)softmax_scale * 1.4426950408889634);
+    if (!isfinite(coef)) return WQ_ERR_SHAPE;  // the scale times post * log2(e) must stay finite in fp32
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int mi = (int)m;
     if (mi <= 1) return tq3_attn::launch<1>(q, q_dtype, heads, mi, k_records, v_records, S, mask, coef, out, out_dtype, s);

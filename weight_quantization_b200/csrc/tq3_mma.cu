@@ -351,7 +351,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t v = (stream + it * n_streams) * kTile + tid;
         int64_t slot = v;  // the slot's load is issued here, ahead of its use at the store
         if constexpr (kLay == tq3::kPool) slot = v < n_vec ? __ldg(static_cast<const int64_t *>(pm.index) + v) : -1;
-        uint8_t *const rec = packed + slot * (kLay == tq3::kSoA ? 48 : 56);
         uint32_t o[12];
         tmem_wait(za);
         tmem_ld32(my_lanes + 32, zb);
@@ -373,11 +372,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (kLay != tq3::kSoA) {  // a 56-byte record is 8-byte aligned
                 if (kLay == tq3::kPool && slot >= pm.n_pool) atomicOr(&g_fault, tq3::kFaultPoolIndex);
                 if (kLay == tq3::kAoS || (slot >= 0 && slot < pm.n_pool)) {
+                    uint8_t *const rec = packed + slot * 56;  // formed only for a slot inside the pool
 #pragma unroll
                     for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
                     st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
                 }
             } else {
+                uint8_t *const rec = packed + v * 48;
                 st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
                 st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
                 st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));

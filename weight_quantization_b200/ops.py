@@ -88,6 +88,17 @@ def _fits(t, n: int, name: str):
         raise ValueError(f"{name} holds {t.numel()} elements; the call needs {n}")
 
 
+def _on(t, device, name: str, dtypes=None):
+    """A caller-supplied buffer must live on the device whose stream the call is enqueued on (the
+    library writes it through a raw pointer from that context) and have a dtype the call takes."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor) or t.device != torch.device(device):
+        raise ValueError(f"{name} must be on {device}")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError(f"{name} must be one of {sorted(str(d) for d in dtypes)}")
+
+
 def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
@@ -126,6 +137,8 @@ def tq3_encode(x: torch.Tensor, sign_mask, packed=None, norms=None, scales=None,
         norms = torch.empty(lead, dtype=torch.float32, device=x.device)
     if scales is None:
         scales = torch.empty(lead, dtype=torch.float32, device=x.device)
+    for name, t in (("packed", packed), ("norms", norms), ("scales", scales)):
+        _on(t, x.device, name)
     _fits(packed, 48 * n_vec, "packed")
     _fits(norms, n_vec, "norms")
     _fits(scales, n_vec, "scales")
@@ -145,6 +158,9 @@ def tq3_decode(packed: torch.Tensor, norms: torch.Tensor, scales: torch.Tensor, 
     n_vec = norms.numel()
     if out is None:
         out = torch.empty(tuple(norms.shape) + (128,), dtype=out_dtype, device=packed.device)
+    for name, t in (("norms", norms), ("scales", scales)):
+        _on(t, packed.device, name)
+    _on(out, packed.device, "out", _DT)
     _fits(out, 128 * n_vec, "out")
     m = _mask_arg(sign_mask)
     st = lib().tq3_decode(_dev(packed, "packed"), _dev(norms, "norms"), _dev(scales, "scales"), n_vec,
@@ -163,6 +179,7 @@ def tq3_encode_aos(x: torch.Tensor, sign_mask, records=None):
     lead = tuple(x.shape[:-1]) + (x.shape[-1] // 128,)
     if records is None:
         records = torch.empty(lead + (56,), dtype=torch.uint8, device=x.device)
+    _on(records, x.device, "records")
     _fits(records, 56 * (x.numel() // 128), "records")
     m = _mask_arg(sign_mask)
     st = lib().tq3_encode_aos(_dev(x, "x"), _DT[x.dtype], x.numel() // 128, m.ctypes.data, _dev(records, "records"),
@@ -178,6 +195,7 @@ def tq3_decode_aos(records: torch.Tensor, sign_mask, out_dtype=torch.float32, ou
     n_vec = records.numel() // 56
     if out is None:
         out = torch.empty(tuple(records.shape[:-1]) + (128,), dtype=out_dtype, device=records.device)
+    _on(out, records.device, "out", _DT)
     _fits(out, 128 * n_vec, "out")
     m = _mask_arg(sign_mask)
     st = lib().tq3_decode_aos(_dev(records, "records"), n_vec, m.ctypes.data, _dev(out, "out"), _DT[out.dtype],
@@ -200,6 +218,8 @@ def tq3_encode_slots(x: torch.Tensor, sign_mask, slots: torch.Tensor, pool: torc
         raise ValueError("slots must be int64 with one entry per vector")
     if pool.dtype != torch.uint8 or pool.ndim != 2 or pool.shape[1] != 56:
         raise ValueError("pool must be uint8 [n_pool, 56]")
+    _on(slots, x.device, "slots")
+    _on(pool, x.device, "pool")
     m = _mask_arg(sign_mask)
     st = lib().tq3_encode_slots(_dev(x, "x"), _DT[x.dtype], n_vec, m.ctypes.data, _dev(slots, "slots"),
                                 _dev(pool, "pool"), pool.shape[0], _stream(x.device))
@@ -219,6 +239,8 @@ def tq3_decode_paged(pool: torch.Tensor, page_table: torch.Tensor, page_size: in
         raise ValueError("page_table must be int32")
     if out is None:
         out = torch.empty((n_vec, 128), dtype=out_dtype, device=pool.device)
+    _on(page_table, pool.device, "page_table")
+    _on(out, pool.device, "out", _DT)
     _fits(out, 128 * n_vec, "out")
     m = _mask_arg(sign_mask)
     st = lib().tq3_decode_paged(_dev(pool, "pool"), pool.shape[0], _dev(page_table, "page_table"),
@@ -243,6 +265,9 @@ def tq3_attention(q: torch.Tensor, k_records: torch.Tensor, v_records: torch.Ten
         raise ValueError("k_records and v_records must have the same shape")
     if out is None:
         out = torch.empty((heads, m, 128), dtype=out_dtype or q.dtype, device=q.device)
+    _on(k_records, q.device, "k_records")
+    _on(v_records, q.device, "v_records")
+    _on(out, q.device, "out", _DT)
     _fits(out, heads * m * 128, "out")
     msk = _mask_arg(sign_mask)
     st = lib().tq3_attention(_dev(q, "q"), _DT[q.dtype], heads, m, _dev(k_records, "k_records"),
@@ -279,6 +304,8 @@ def rpbh_quantize_weight(W: torch.Tensor, perm: torch.Tensor, signs: torch.Tenso
         packed = torch.empty(max(rpbh_packed_bytes(rows, d, bits), 0), dtype=torch.uint8, device=W.device)
     if row_norms is None:
         row_norms = torch.empty(rows, dtype=W.dtype, device=W.device)
+    for name, t in (("packed", packed), ("row_norms", row_norms), ("perm", perm), ("signs", signs)):
+        _on(t, W.device, name)
     _fits(packed, rpbh_packed_bytes(rows, d, bits), "packed")
     _fits(row_norms, rows, "row_norms")
     _fits(perm, d, "perm")
@@ -296,6 +323,9 @@ def rpbh_dequantize_weight(packed: torch.Tensor, row_norms: torch.Tensor, rows: 
     cb = _codebook_arg(codebook, bits)
     if out is None:
         out = torch.empty(rows, d, dtype=out_dtype, device=packed.device)
+    for name, t in (("row_norms", row_norms), ("perm", perm), ("signs", signs)):
+        _on(t, packed.device, name)
+    _on(out, packed.device, "out", _DT)
     _fits(packed, rpbh_packed_bytes(rows, d, bits), "packed")
     _fits(row_norms, rows, "row_norms")
     _fits(out, rows * d, "out")
@@ -316,6 +346,9 @@ def rpbh_rotate_activations(x: torch.Tensor, perm: torch.Tensor, signs: torch.Te
     rows, d = x.shape
     if out is None:
         out = torch.empty_like(x)
+    for name, t in (("perm", perm), ("signs", signs)):
+        _on(t, x.device, name)
+    _on(out, x.device, "out", (x.dtype,))
     _fits(out, rows * d, "out")
     _fits(perm, d, "perm")
     _fits(signs, d, "signs")
@@ -332,6 +365,9 @@ def rpbh_linear(packed: torch.Tensor, row_norms: torch.Tensor, out_features: int
     m = x_rot.shape[0]
     if out is None:
         out = torch.empty(m, out_features, dtype=torch.bfloat16, device=x_rot.device)
+    for name, t in (("packed", packed), ("row_norms", row_norms), ("bias", bias)):
+        _on(t, x_rot.device, name)
+    _on(out, x_rot.device, "y", (torch.bfloat16,))
     _fits(packed, rpbh_packed_bytes(out_features, d, bits), "packed")
     _fits(row_norms, out_features, "row_norms")
     _fits(x_rot, m * d, "x_rot")
