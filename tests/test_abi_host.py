@@ -111,6 +111,10 @@ def test_lloyd_max_host_helper_matches_oracle(wq, oracle):
     for bits in (2, 3, 4):
         for d in (32, 96, 3072, 11008):
             assert np.array_equal(wq.rpbh_codebook(bits, d), oracle.rpbh_codebook(bits, d))
+    from conftest import read_golden
+    for parts in read_golden("lloyd_max_fp32.txt"):  # and against the independent fp32 bit patterns
+        want = np.array([int(v, 16) for v in parts[1:]], dtype=np.uint32)
+        assert np.array_equal(wq.gaussian_lloyd_max(int(parts[0])).view(np.uint32), want)
     with pytest.raises(wq.WQError):
         wq.gaussian_lloyd_max(5)
     with pytest.raises(wq.WQError):
@@ -204,3 +208,37 @@ def test_bindings_reject_buffers_smaller_than_the_call(wq):
         wq.rpbh_dequantize_weight(torch.zeros(95, dtype=torch.uint8), torch.zeros(4), 4, 64, 3, cb)
     with pytest.raises(ValueError, match="row_norms holds"):
         wq.rpbh_linear(torch.zeros(96, dtype=torch.uint8), torch.zeros(3), 4, 64, 3, cb, torch.zeros(2, 64))
+
+
+def test_bindings_reject_buffers_on_another_device_or_dtype(wq):
+    """A caller-supplied buffer is written through a raw pointer on the stream of the call's main
+    operand, so the binding rejects one that lives on another device or has a dtype the call does
+    not take ("meta" tensors stand in for a second device on a CPU-only host)."""
+    mask = np.zeros(4, np.uint32)
+    rec = torch.zeros(2, 10, 56, dtype=torch.uint8)
+    q = torch.zeros(2, 4, 128)
+    with pytest.raises(ValueError, match="out must be on"):
+        wq.tq3_attention(q, rec, rec, mask, out=torch.empty(2, 4, 128, device="meta"))
+    with pytest.raises(ValueError, match="out must be one of"):
+        wq.tq3_attention(q, rec, rec, mask, out=torch.empty(2, 4, 128, dtype=torch.int32))
+    with pytest.raises(ValueError, match="k_records must be on"):
+        wq.tq3_attention(q, rec.to("meta"), rec, mask)
+    pool, table = torch.zeros(64, 56, dtype=torch.uint8), torch.zeros(4, dtype=torch.int32)
+    with pytest.raises(ValueError, match="out must be on"):
+        wq.tq3_decode_paged(pool, table, 16, 64, mask, out=torch.empty(64, 128, device="meta"))
+    with pytest.raises(ValueError, match="out must be one of"):
+        wq.tq3_decode_paged(pool, table, 16, 64, mask, out=torch.empty(64, 128, dtype=torch.float16))
+    with pytest.raises(ValueError, match="page_table must be on"):
+        wq.tq3_decode_paged(pool, table.to("meta"), 16, 64, mask)
+    p, n, s = torch.zeros(4, 48, dtype=torch.uint8), torch.zeros(4), torch.zeros(4)
+    with pytest.raises(ValueError, match="out must be on"):
+        wq.tq3_decode(p, n, s, mask, out=torch.empty(4, 128, device="meta"))
+    with pytest.raises(ValueError, match="norms must be on"):
+        wq.tq3_decode(p, n.to("meta"), s, mask)
+    with pytest.raises(ValueError, match="packed must be on"):
+        wq.tq3_encode(torch.zeros(4, 128), mask, packed=torch.empty(4, 48, dtype=torch.uint8, device="meta"))
+    perm, signs = torch.zeros(64, dtype=torch.int32), torch.ones(64, dtype=torch.int8)
+    with pytest.raises(ValueError, match="out must be one of"):
+        wq.rpbh_rotate_activations(torch.zeros(4, 64), perm, signs, out=torch.empty(4, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="perm must be on"):
+        wq.rpbh_rotate_activations(torch.zeros(4, 64), perm.to("meta"), signs)

@@ -367,6 +367,30 @@ def test_lloyd_max_fixed_point_by_quadrature(oracle):
             assert abs(m1 / m0 - c[k]) < tol, (bits, k, m1 / m0, c[k])
 
 
+def test_lloyd_max_fp32_bits_exact(oracle):
+    """The fp32 codebooks of gaussian_lloyd_max(bits, iters=200), bit for bit, against values
+    computed by an independent float64 implementation of the page's iteration. At 4 bits the
+    iterate still moves by about 1.8e-5 per step, so 199 or 201 iterations must differ in every
+    level: this catches an off-by-one iteration count that the 1e-3 / 1e-4 checks above allow."""
+    seen = set()
+    for parts in read_golden("lloyd_max_fp32.txt"):
+        bits = int(parts[0])
+        want = np.array([int(v, 16) for v in parts[1:]], dtype=np.uint32)
+        assert want.size == 1 << bits
+        got = oracle.gaussian_lloyd_max(bits).view(np.uint32)
+        assert np.array_equal(got, want), (bits, [f"{v:08x}" for v in got])
+        seen.add(bits)
+    assert seen == {2, 3, 4}
+    c200 = oracle.gaussian_lloyd_max(4, 200)
+    for iters in (199, 201):
+        other = oracle.gaussian_lloyd_max(4, iters)
+        assert np.all(other != c200), iters
+        assert np.abs(other.astype(np.float64) - c200).max() < 5e-5
+    for bits in (2, 3):  # fp32 fixed points: one more or one fewer step changes nothing
+        assert np.array_equal(oracle.gaussian_lloyd_max(bits, 199), oracle.gaussian_lloyd_max(bits, 200))
+        assert np.array_equal(oracle.gaussian_lloyd_max(bits, 201), oracle.gaussian_lloyd_max(bits, 200))
+
+
 def test_rpbh_codebook_scaling(oracle):
     for bits in (2, 3, 4):
         for d in (3072, 11008):
