@@ -60,6 +60,64 @@ __host__ __device__ __forceinline__ float centroid(uint32_t idx) {
     return (idx & 4u) ? mag : -mag;
 }
 
+// The page's steps for one vector, one IEEE fp32 operation at a time, by a single thread from
+// global memory (tq3_quantize steps 1-6): n = max(fp32(sqrt(sum x^2 in fp64, index order)), 1e-8),
+// xn = x / n, the sign flips, the seven butterfly stages h = 1 .. 64 and the post-multiplier,
+// s = max(max|xh|, 1e-8), xs = xh / s, the index #{j : B_j < xs}, _pack_3bit. The fast encoders
+// transform the unnormalised vector, which overflows fp32 once sum |x| passes FLT_MAX (a finite
+// input whose normalised form the page encodes without trouble); a vector whose fp32 sum of
+// squares is not finite is re-encoded here instead. It runs rarely (|x| beyond about 1e18), so it
+// keeps its vector in local memory and costs the caller no registers. Writes the 48 packed bytes
+// at rec (byte stores), the norm and the scale.
+static __device__ __noinline__ void encode_vector_exact(const void *x, bool x_bf16, int64_t v, const SignMask &mask,
+                                                        uint8_t *rec, float *norm_out, float *scale_out) {
+    float y[kD];
+#pragma unroll 1
+    for (int i = 0; i < kD; ++i)
+        y[i] = x_bf16 ? __uint_as_float((uint32_t)static_cast<const uint16_t *>(x)[v * kD + i] << 16)
+                      : static_cast<const float *>(x)[v * kD + i];
+    double ss = 0.0;
+#pragma unroll 1
+    for (int i = 0; i < kD; ++i) ss = __dadd_rn(ss, __dmul_rn((double)y[i], (double)y[i]));
+    const float n = fmaxf(__double2float_rn(__dsqrt_rn(ss)), 1e-8f);
+#pragma unroll 1
+    for (int i = 0; i < kD; ++i) {
+        const uint32_t flip = ((mask.w[i >> 5] >> (i & 31)) & 1u) ? 0u : 0x80000000u;
+        y[i] = __uint_as_float(__float_as_uint(__fdiv_rn(y[i], n)) ^ flip);
+    }
+#pragma unroll 1
+    for (int h = 1; h < kD; h <<= 1)
+#pragma unroll 1
+        for (int i = 0; i < kD; ++i)
+            if ((i & h) == 0) {
+                const float a = y[i], b = y[i + h];
+                y[i] = __fadd_rn(a, b);
+                y[i + h] = __fsub_rn(a, b);
+            }
+    float s = 0.0f;
+#pragma unroll 1
+    for (int i = 0; i < kD; ++i) {
+        y[i] = __fmul_rn(y[i], fwht_post());
+        s = fabsf(y[i]) > s ? fabsf(y[i]) : s;
+    }
+    s = s < 1e-8f ? 1e-8f : s;
+#pragma unroll 1
+    for (int g = 0; g < 16; ++g) {
+        uint32_t bits = 0;
+        for (int e = 0; e < 8; ++e) {
+            const float xs = __fdiv_rn(y[8 * g + e], s);
+            const uint32_t idx = (xs > -0.7992f) + (xs > -0.4824f) + (xs > -0.2304f) + (xs > 0.0f) +
+                                 (xs > 0.2304f) + (xs > 0.4824f) + (xs > 0.7992f);
+            bits |= idx << (3 * e);
+        }
+        rec[3 * g] = (uint8_t)bits;
+        rec[3 * g + 1] = (uint8_t)(bits >> 8);
+        rec[3 * g + 2] = (uint8_t)(bits >> 16);
+    }
+    *norm_out = n;
+    *scale_out = s;
+}
+
 __device__ __forceinline__ unsigned char *tile_base(unsigned char *raw) {
     return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
 }

@@ -16,7 +16,10 @@
 // Numerics: the fp32 accumulation order of the tensor core is not the butterfly's, so z agrees
 // with the step-by-step transform to a few units in the last place relative to max|z|; as for the
 // CUDA-core fast encoder, an index can differ from the page's rounding only for a coefficient
-// within about 1e-6 of a boundary. Norms and scales agree to within 1e-6 relative.
+// within about 1e-6 of a boundary. Norms and scales agree to within 1e-6 relative. A vector whose
+// fp32 sum of squares is not finite (|x| beyond about 1e19, where the unnormalised product can
+// itself overflow although the page's normalised transform does not) is re-encoded by the page's
+// steps from global memory (tq3::encode_vector_exact).
 //
 // Pipeline per CTA (persistent over tiles): TMA load of the next tile is issued as soon as the
 // tensor core has consumed the current one, so it lands while the 128 threads run the epilogue;
@@ -197,8 +200,8 @@ __device__ __align__(128) const BTable kDefaultB = make_default_b();
 // pool at `packed` (a negative slot: not stored). Norms and scales are unused for the record layouts.
 template <bool kFold, int kLay = tq3::kSoA>
 __global__ void __launch_bounds__(kThreads, 1)
-    encode_mma(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, SignMask mask, uint8_t *__restrict__ packed,
-               float *__restrict__ norms, float *__restrict__ scales, tq3::PoolMap pm) {
+    encode_mma(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, const void *__restrict__ x, SignMask mask,
+               uint8_t *__restrict__ packed, float *__restrict__ norms, float *__restrict__ scales, tq3::PoolMap pm) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *const base = tq3::tile_base(smem_raw);
     const int grp = threadIdx.x >> 7, tid = threadIdx.x & 127, warp = tid >> 5;
@@ -322,23 +325,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             n2 = __fadd_rn(a0, a1);
         }
         const float m = fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3]));
-        float nrm0 = __fsqrt_rn(__fmul_rn(n2, 0.0078125f));
-        // the fp32 squares overflowed: sum them in fp64 (taken by the whole warp, since the
-        // accumulator reads are warp-collective; lanes that do not need it discard the result)
+        // A vector whose fp32 squares overflowed (|x| beyond about 1e19; z itself may have
+        // overflowed) still takes part in the warp-collective accumulator reads below, and is then
+        // re-encoded step by step at the store.
         const bool big = !(n2 <= 3.0e38f);
-        if (__any_sync(0xffffffffu, big)) {
-            double d = 0.0;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float z[32];
-                tmem_ld32(my_lanes + 32 * c, z);
-                tmem_wait(z);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) d = __fma_rn((double)z[i], (double)z[i], d);
-            }
-            if (big) nrm0 = __double2float_rn(__dsqrt_rn(d * 0.0078125));
-        }
-        const float nrm = fmaxf(nrm0, 1e-8f);
+        const float nrm = fmaxf(__fsqrt_rn(__fmul_rn(n2, 0.0078125f)), 1e-8f);
         const float sraw = __fmul_rn(__fdiv_rn(m, nrm), post);
         const float scale = fmaxf(sraw, 1e-8f);
         const float T = (sraw >= 1e-8f) ? m : __fmul_rn(__fmul_rn(1e-8f, nrm), 11.3137085f);
@@ -373,17 +364,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (kLay == tq3::kPool && slot >= pm.n_pool) atomicOr(&g_fault, tq3::kFaultPoolIndex);
                 if (kLay == tq3::kAoS || (slot >= 0 && slot < pm.n_pool)) {
                     uint8_t *const rec = packed + slot * 56;  // formed only for a slot inside the pool
+                    if (big) {
+                        tq3::encode_vector_exact(x, true, v, mask, rec, reinterpret_cast<float *>(rec + 48),
+                                                 reinterpret_cast<float *>(rec + 52));
+                    } else {
 #pragma unroll
-                    for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
-                    st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+                        for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
+                        st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+                    }
                 }
             } else {
                 uint8_t *const rec = packed + v * 48;
-                st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
-                st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
-                st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));
-                norms[v] = nrm;
-                scales[v] = scale;
+                if (big) {
+                    tq3::encode_vector_exact(x, true, v, mask, rec, norms + v, scales + v);
+                } else {
+                    st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
+                    st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
+                    st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));
+                    norms[v] = nrm;
+                    scales[v] = scale;
+                }
             }
         }
     }
@@ -416,15 +416,15 @@ int sm_count() {
 }
 
 template <typename K>
-wq_status launch(K k, int64_t cnt, const CUtensorMap &tm, const SignMask &m, uint8_t *pc, float *nc, float *sc,
-                 const tq3::PoolMap &pm, cudaStream_t s) {
+wq_status launch(K k, int64_t cnt, const CUtensorMap &tm, const void *xc, const SignMask &m, uint8_t *pc, float *nc,
+                 float *sc, const tq3::PoolMap &pm, cudaStream_t s) {
     if (!ensure_dynamic_smem(reinterpret_cast<const void *>(k), kSmem)) return WQ_ERR_CUDA;
     // one CTA per SM (it holds all 512 tensor-memory columns), never more CTAs than tile triples
     const int64_t tiles = (cnt + kTile - 1) / kTile;
     const int64_t triples = (tiles + kGroups - 1) / kGroups;
     const int64_t g_ = sm_count() > 0 ? sm_count() : 1;
     const int64_t g = g_ < triples ? g_ : triples;
-    if (launch_pdl(k, (unsigned)g, kThreads, kSmem, s, cnt, tm, m, pc, nc, sc, pm) != cudaSuccess) {
+    if (launch_pdl(k, (unsigned)g, kThreads, kSmem, s, cnt, tm, xc, m, pc, nc, sc, pm) != cudaSuccess) {
         cudaGetLastError();
         return WQ_ERR_CUDA;
     }
@@ -445,16 +445,16 @@ wq_status encode_bf16(const void *x, int64_t n_vec, const SignMask &m, uint8_t *
         if (layout == tq3::kPool) {  // the pool is not offset; the chunk's slots are
             tq3::PoolMap pm = pool;
             pm.index = static_cast<const int64_t *>(pool.index) + off;
-            st = def ? launch(encode_mma<true, tq3::kPool>, cnt, tm, m, packed, nullptr, nullptr, pm, s)
-                     : launch(encode_mma<false, tq3::kPool>, cnt, tm, m, packed, nullptr, nullptr, pm, s);
+            st = def ? launch(encode_mma<true, tq3::kPool>, cnt, tm, xc, m, packed, nullptr, nullptr, pm, s)
+                     : launch(encode_mma<false, tq3::kPool>, cnt, tm, xc, m, packed, nullptr, nullptr, pm, s);
         } else if (layout == tq3::kAoS) {
             uint8_t *const pc = packed + off * 56;
-            st = def ? launch(encode_mma<true, tq3::kAoS>, cnt, tm, m, pc, nullptr, nullptr, pool, s)
-                     : launch(encode_mma<false, tq3::kAoS>, cnt, tm, m, pc, nullptr, nullptr, pool, s);
+            st = def ? launch(encode_mma<true, tq3::kAoS>, cnt, tm, xc, m, pc, nullptr, nullptr, pool, s)
+                     : launch(encode_mma<false, tq3::kAoS>, cnt, tm, xc, m, pc, nullptr, nullptr, pool, s);
         } else {
             uint8_t *const pc = packed + off * 48;
-            st = def ? launch(encode_mma<true>, cnt, tm, m, pc, norms + off, scales + off, pool, s)
-                     : launch(encode_mma<false>, cnt, tm, m, pc, norms + off, scales + off, pool, s);
+            st = def ? launch(encode_mma<true>, cnt, tm, xc, m, pc, norms + off, scales + off, pool, s)
+                     : launch(encode_mma<false>, cnt, tm, xc, m, pc, norms + off, scales + off, pool, s);
         }
         if (st != WQ_OK) return st;
     }

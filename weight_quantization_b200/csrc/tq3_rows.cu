@@ -21,7 +21,10 @@
 // fp32 values it compares; the only difference from the page's own rounding sequence is a few
 // units in the last place of xs, so an index can differ from the step-by-step result only for a
 // coefficient within about 1e-6 of a boundary (ties included). Norms come from an fp32 sum of
-// squares (within 1e-6 relative), scales = max(RN(RN(max|z| / norm) * c), 1e-8).
+// squares (within 1e-6 relative), scales = max(RN(RN(max|z| / norm) * c), 1e-8). A vector whose
+// fp32 sum of squares is not finite (|x| beyond about 1e19, where the unnormalised transform can
+// itself overflow although the page's normalised one does not) is encoded by the page's steps
+// instead, from global memory (tq3::encode_vector_exact).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -113,8 +116,8 @@ __device__ __forceinline__ float edge(int k) { return k == 0 ? 0.2304f : k == 1 
 // decode_rows, norms and scales are unused for the record layouts).
 template <bool kBf16, bool kFold, int kLay = tq3::kSoA>
 __global__ void __launch_bounds__(kThreads, kMinBlocks)
-    encode_rows(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, SignMask mask, uint8_t *__restrict__ packed,
-                float *__restrict__ norms, float *__restrict__ scales, tq3::PoolMap pm) {
+    encode_rows(int64_t n_vec, const __grid_constant__ CUtensorMap tmap, const void *__restrict__ x, SignMask mask,
+                uint8_t *__restrict__ packed, float *__restrict__ norms, float *__restrict__ scales, tq3::PoolMap pm) {
     using G = EncGeo<kBf16>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *const base = tq3::tile_base(smem_raw);
@@ -246,21 +249,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         }
         const float m = fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3]));
 
-        // norm, scale and the |z| thresholds
-        float nrm0 = __fsqrt_rn(n2);
-        if (!(n2 <= 3.0e38f)) {
-            // the fp32 squares overflowed (|x| beyond ~1e19): ||x||^2 = ||z||^2 / 128, in fp64
-            double d = 0.0;
-#pragma unroll
-            for (int k = 0; k < 64; ++k) {
-                float a, b;
-                upk2(P[k], a, b);
-                d = __fma_rn((double)a, (double)a, d);
-                d = __fma_rn((double)b, (double)b, d);
-            }
-            nrm0 = __double2float_rn(__dsqrt_rn(d * 0.0078125));
-        }
-        const float nrm = fmaxf(nrm0, 1e-8f);
+        // norm, scale and the |z| thresholds. A vector whose fp32 squares overflowed (|x| beyond
+        // about 1e19; z itself may have overflowed) is re-encoded step by step at the store below.
+        const bool big = !(n2 <= 3.0e38f);
+        const float nrm = fmaxf(__fsqrt_rn(n2), 1e-8f);
         const float sraw = __fmul_rn(__fdiv_rn(m, nrm), post);
         const float scale = fmaxf(sraw, 1e-8f);
         const float T = (sraw >= 1e-8f) ? m : __fmul_rn(__fmul_rn(1e-8f, nrm), 11.3137085f);
@@ -323,17 +315,26 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
                 if (kLay == tq3::kPool && slot >= pm.n_pool) atomicOr(&g_fault, tq3::kFaultPoolIndex);
                 if (kLay == tq3::kAoS || (slot >= 0 && slot < pm.n_pool)) {
                     uint8_t *rec = packed + slot * 56;
+                    if (big) {
+                        tq3::encode_vector_exact(x, kBf16, v, mask, rec, reinterpret_cast<float *>(rec + 48),
+                                                 reinterpret_cast<float *>(rec + 52));
+                    } else {
 #pragma unroll
-                    for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
-                    st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+                        for (int q = 0; q < 6; ++q) st_stream8(rec + 8 * q, make_uint2(o[2 * q], o[2 * q + 1]));
+                        st_stream8(rec + 48, make_uint2(__float_as_uint(nrm), __float_as_uint(scale)));
+                    }
                 }
             } else {
                 uint8_t *rec = packed + v * 48;
-                st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
-                st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
-                st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));
-                norms[v] = nrm;
-                scales[v] = scale;
+                if (big) {
+                    tq3::encode_vector_exact(x, kBf16, v, mask, rec, norms + v, scales + v);
+                } else {
+                    st_stream16(rec, make_uint4(o[0], o[1], o[2], o[3]));
+                    st_stream16(rec + 16, make_uint4(o[4], o[5], o[6], o[7]));
+                    st_stream16(rec + 32, make_uint4(o[8], o[9], o[10], o[11]));
+                    norms[v] = nrm;
+                    scales[v] = scale;
+                }
             }
         }
     }
@@ -574,22 +575,23 @@ int grid_for(K k, size_t smem, int64_t tiles) {
 }
 
 template <typename K>
-wq_status launch_enc(K k, size_t smem, int64_t cnt, const CUtensorMap &tm, const SignMask &m, uint8_t *pc, float *nc,
-                     float *sc, const tq3::PoolMap &pm, cudaStream_t s) {
+wq_status launch_enc(K k, size_t smem, int64_t cnt, const CUtensorMap &tm, const void *xc, const SignMask &m,
+                     uint8_t *pc, float *nc, float *sc, const tq3::PoolMap &pm, cudaStream_t s) {
     if (!ensure_dynamic_smem(reinterpret_cast<const void *>(k), smem)) return WQ_ERR_CUDA;
     const int64_t tiles = (cnt + kTile - 1) / kTile;
-    k<<<grid_for(k, smem, tiles), kThreads, smem, s>>>(cnt, tm, m, pc, nc, sc, pm);
+    k<<<grid_for(k, smem, tiles), kThreads, smem, s>>>(cnt, tm, xc, m, pc, nc, sc, pm);
     return launch_status();
 }
 
 template <int kLay>
-wq_status launch_enc_lay(bool bf, bool def, size_t smem, int64_t cnt, const CUtensorMap &tm, const SignMask &m,
-                         uint8_t *pc, float *nc, float *sc, const tq3::PoolMap &pm, cudaStream_t s) {
+wq_status launch_enc_lay(bool bf, bool def, size_t smem, int64_t cnt, const CUtensorMap &tm, const void *xc,
+                         const SignMask &m, uint8_t *pc, float *nc, float *sc, const tq3::PoolMap &pm,
+                         cudaStream_t s) {
     if (bf)
-        return def ? launch_enc(encode_rows<true, true, kLay>, smem, cnt, tm, m, pc, nc, sc, pm, s)
-                   : launch_enc(encode_rows<true, false, kLay>, smem, cnt, tm, m, pc, nc, sc, pm, s);
-    return def ? launch_enc(encode_rows<false, true, kLay>, smem, cnt, tm, m, pc, nc, sc, pm, s)
-               : launch_enc(encode_rows<false, false, kLay>, smem, cnt, tm, m, pc, nc, sc, pm, s);
+        return def ? launch_enc(encode_rows<true, true, kLay>, smem, cnt, tm, xc, m, pc, nc, sc, pm, s)
+                   : launch_enc(encode_rows<true, false, kLay>, smem, cnt, tm, xc, m, pc, nc, sc, pm, s);
+    return def ? launch_enc(encode_rows<false, true, kLay>, smem, cnt, tm, xc, m, pc, nc, sc, pm, s)
+               : launch_enc(encode_rows<false, false, kLay>, smem, cnt, tm, xc, m, pc, nc, sc, pm, s);
 }
 
 wq_status encode(const void *x, int x_dtype, int64_t n_vec, const SignMask &m, uint8_t *packed, float *norms,
@@ -608,12 +610,13 @@ wq_status encode(const void *x, int x_dtype, int64_t n_vec, const SignMask &m, u
         if (layout == tq3::kPool) {  // the pool is not offset; the chunk's slots are
             tq3::PoolMap pm = pool;
             pm.index = static_cast<const int64_t *>(pool.index) + off;
-            st = launch_enc_lay<tq3::kPool>(bf, def, smem, cnt, tm, m, packed, nullptr, nullptr, pm, s);
+            st = launch_enc_lay<tq3::kPool>(bf, def, smem, cnt, tm, xc, m, packed, nullptr, nullptr, pm, s);
         } else if (layout == tq3::kAoS) {
-            st = launch_enc_lay<tq3::kAoS>(bf, def, smem, cnt, tm, m, packed + off * 56, nullptr, nullptr, pool, s);
+            st = launch_enc_lay<tq3::kAoS>(bf, def, smem, cnt, tm, xc, m, packed + off * 56, nullptr, nullptr, pool,
+                                           s);
         } else {
-            st = launch_enc_lay<tq3::kSoA>(bf, def, smem, cnt, tm, m, packed + off * 48, norms + off, scales + off,
-                                           pool, s);
+            st = launch_enc_lay<tq3::kSoA>(bf, def, smem, cnt, tm, xc, m, packed + off * 48, norms + off,
+                                           scales + off, pool, s);
         }
         if (st != WQ_OK) return st;
     }
