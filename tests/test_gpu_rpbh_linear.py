@@ -68,9 +68,11 @@ def test_linear_norm_dtype_and_bias(wq, oracle, norm_bf16, with_bias):
 
 
 def test_linear_llm_full_size_sampled_rows(wq, oracle):
-    """W[4096, 11008] at 3 bits times x_rot[2048, 11008]: every output of 48 sampled activation rows."""
-    rows = np.random.default_rng(5).choice(2048, size=48, replace=False)
-    _case(wq, oracle, 4096, 11008, 2048, 3, norm_bf16=True, with_bias=True, seed=42, check_rows=np.sort(rows))
+    """W[4096, 11008] at 3 bits times x_rot[2048, 11008]: every output of 264 activation rows (every
+    eighth row, which touches each of the kernel's 256-row tiles 32 times, plus the first and last
+    rows of every tile), against the fp64 oracle."""
+    rows = np.unique(np.concatenate([np.arange(0, 2048, 8), np.arange(0, 2048, 256) + 255]))
+    _case(wq, oracle, 4096, 11008, 2048, 3, norm_bf16=True, with_bias=True, seed=42, check_rows=rows)
 
 
 def test_linear_errors(wq):

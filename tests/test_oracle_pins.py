@@ -613,3 +613,19 @@ def test_tq3_dot_products_in_the_indices_basis(oracle):
     direct_v = w @ k
     rotated_v = s * (H @ ((w * coef) @ cv))
     assert np.abs(direct_v - rotated_v).max() <= 1e-5 * np.abs(w).sum() * np.abs(k).max()
+
+
+def test_tq3_tie_counts_of_the_round_trip_workload(oracle):
+    """The stored oracle counts for the 4096-vector round trip (tests/golden/tq3_tie_counts.txt)
+    still hold: 352 exact zeros, all from the 32 constant blocks (11 each, the pre-flip pin above),
+    inside 649 coefficients within 1e-6 of a boundary."""
+    from weight_quantization_b200 import inputs
+    want = {r[0]: tuple(int(v) for v in r[1:]) for r in read_golden("tq3_tie_counts.txt")}
+    x = inputs.tq3_roundtrip()
+    xs, _, _, _ = oracle.tq3_encode_debug(x, inputs.tq3_sign_bits())
+    _, B = oracle.tq3_tables()
+    near = np.zeros(xs.shape, bool)
+    for b in B.astype(np.float64):
+        near |= np.abs(xs.astype(np.float64) - b) < 1e-6
+    assert (xs.shape[0], int(near.sum()), int((xs == 0).sum())) == want["tq3_roundtrip_fp32"]
+    assert int((xs[4064:] == 0).sum()) == 32 * 11 == want["tq3_roundtrip_fp32"][2]
