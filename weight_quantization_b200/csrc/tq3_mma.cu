@@ -7,16 +7,16 @@
 // and s the sign flips: z_j = -fwht(s x)_j. Every product is exact (a bf16 value times +-1) and
 // the sums accumulate in fp32 in tensor memory; one tcgen05.mma per 16 columns of K, issued by a
 // single thread, eight per tile. Thread t of the CTA then owns vector t: it reads row t of the
-// accumulator (tcgen05.ld, its warp's 32-lane quarter) into 128 registers and runs the same
-// decision and packing as the CUDA-core fast encoder (norm from ||z||^2 / 128, absmax T, the
-// index as 3.5 + sgn(-z) (c + 1/2) with c = #{k : |z| > edge_k T}, 8^j-weighted fp32 words).
-// The negation in B makes an exact zero come out as z = +0, i.e. a true -0, whose index is 3 as
-// the page's searchsorted gives for 0.
+// accumulator (tcgen05.ld, its warp's 32-lane quarter) in 32-column pieces, twice: the norm
+// (||z||^2 / 128) and absmax T, then the indices, each from the scaled coefficient x = -z / T as
+// 3 + ceil(Q(x)) with Q an odd quintic through the boundaries (bucket_piece), packed through
+// 8^j-weighted fp32 words. An exact zero coefficient gets index 3, as the page's searchsorted gives.
 //
 // Numerics: the fp32 accumulation order of the tensor core is not the butterfly's, so z agrees
-// with the step-by-step transform to a few units in the last place relative to max|z|; as for the
-// CUDA-core fast encoder, an index can differ from the page's rounding only for a coefficient
-// within about 1e-6 of a boundary. Norms and scales agree to within 1e-6 relative. A vector whose
+// with the step-by-step transform to a few units in the last place relative to max|z|, and the
+// decision polynomial places each boundary within about 1.3e-7 of its exact position; an index can
+// therefore differ from the page's rounding only for a coefficient within about 1e-6 of a
+// boundary. Norms and scales agree to within 1e-6 relative. A vector whose
 // fp32 sum of squares is not finite (|x| beyond about 1e19, where the unnormalised product can
 // itself overflow although the page's normalised transform does not) is re-encoded by the page's
 // steps from global memory (tq3::encode_vector_exact).
@@ -82,21 +82,6 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
     return old;
 }
 
-// (a & b) | c and (a & b) ^ c as single three-input logic operations.
-__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-__device__ __forceinline__ uint32_t lop3_and_xor(uint32_t a, uint32_t b, uint32_t c) {
-    uint32_t d;
-    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-    return d;
-}
-
-// The positive TQ3_BOUNDARIES (fp32).
-__device__ __forceinline__ float edge(int k) { return k == 0 ? 0.2304f : k == 1 ? 0.4824f : 0.7992f; }
-
 // Chunks c0 .. c0 + 3 of row n of B = -H diag(s), K-major with the 128-byte swizzle (two 64-column
 // halves): entry (n, k) is -(-1)^popc(n & k) s_k, exactly +-1 in bf16.
 template <bool kFold>
@@ -123,36 +108,50 @@ __device__ __forceinline__ void build_b(unsigned char *B, const SignMask &mask, 
     }
 }
 
+// fma.rp.f32x2: two fused multiply-adds rounded towards +infinity.
+__device__ __forceinline__ f32x2 fma2_rp(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 r;
+    asm("fma.rp.f32x2 %0,%1,%2,%3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// The decision polynomial. With x = xs the scaled coefficient in [-1, 1], the page's index is
+// #{j : B_j < x} over TQ3_BOUNDARIES B = (-b2, -b1, -b0, 0, b0, b1, b2). Let Q be the odd quintic
+// Q(x) = q1 x + q3 x^3 + q5 x^5 with Q(b_k) = k + 1 for the three positive boundaries (solved in
+// fp64 from the fp32 boundary values, then rounded to fp32). Q is increasing on [-1, 1] (Q' >= 1.97)
+// and Q(1) = 3.46 < 4, so #{j : B_j < x} = 3 + ceil(Q(x)) for every x in [-1, 1]: at a boundary
+// ceil(Q) is exactly the integer k + 1, which puts the value in the lower bucket as searchsorted
+// does, and an exact 0 gives index 3. The ceiling costs nothing: the last Horner step
+// h x + (2^23 + 4) is one fma rounded towards +infinity, whose result (between 2^23 and 2^24) is the
+// integer 2^23 + 4 + ceil(h x). The fp32 evaluation moves each boundary by at most about 1.3e-7 in
+// x, which the parity rule's 1e-6 tie window absorbs.
+__device__ __forceinline__ float q_coef(int k) {
+    return __uint_as_float(k == 1 ? 0x408cce16u : k == 3 ? 0xbf91bb0au : 0x3e4acae9u);
+}
+
 // Indices of one 32-column piece (elements 32c .. 32c + 31, groups 4c .. 4c + 3) packed as the
 // record's bytes 12c .. 12c + 11, three little-endian words (_pack_3bit: group i is bytes
-// 3i .. 3i + 2).
-// Group q is accumulated as two fp32 words, even slots and odd slots, each starting from
-// sum_j 3.5 * 8^j over its slots; each step adds +-8^j (c + 1/2), an integer except for slot 0
-// (+-1/2), which comes first, so every partial sum is an integer below 2^24 and the words are exact.
-__device__ __forceinline__ void bucket_piece(const float (&z)[32], uint32_t Mb, float K0, float K1, float K2,
-                                             uint32_t &o0, uint32_t &o1, uint32_t &o2) {
-    const f32x2 HALF = pk2(0.5f, 0.5f);
+// 3i .. 3i + 2). nr = -1 / T turns the accumulator's z = -fwht into x = z * nr. Group q is
+// accumulated as two fp32 words, even slots and odd slots, each a sum of index * 8^j: integers
+// below 2^24, so the words are exact.
+__device__ __forceinline__ void bucket_piece(const float (&z)[32], float nr, uint32_t &o0, uint32_t &o1, uint32_t &o2) {
+    const f32x2 NR = pk2(nr, nr);
+    const f32x2 Q1 = pk2(q_coef(1), q_coef(1)), Q3 = pk2(q_coef(3), q_coef(3)), Q5 = pk2(q_coef(5), q_coef(5));
+    const f32x2 KK = pk2(8388612.0f, 8388612.0f), NC = pk2(-8388609.0f, -8388609.0f);
     f32x2 W[4];
 #pragma unroll
-    for (int gg = 0; gg < 4; ++gg) W[gg] = pk2(932067.5f, 7456540.0f);
+    for (int gg = 0; gg < 4; ++gg) W[gg] = 0ull;
 #pragma unroll
     for (int p = 0; p < 4; ++p)
 #pragma unroll
         for (int gg = 0; gg < 4; ++gg) {
             const int i = 4 * gg + p;  // local elements 2i (slot 2p) and 2i + 1 (slot 2p + 1)
-            const float za = z[2 * i], zb = z[2 * i + 1];
-            const uint32_t wa = 0x80000000u | ((127u + 6u * p) << 23);      // -8^(2p)
-            const uint32_t wb = 0x80000000u | ((127u + 6u * p + 3u) << 23);  // -8^(2p+1)
-            // copysign(M, z) and copysign(8^j, -z), one three-input logic operation each
-            const float sMa = __uint_as_float(lop3_and_or(__float_as_uint(za), 0x80000000u, Mb));
-            const float sMb = __uint_as_float(lop3_and_or(__float_as_uint(zb), 0x80000000u, Mb));
-            const f32x2 w2 = pk2(__uint_as_float(lop3_and_xor(__float_as_uint(za), 0x80000000u, wa)),
-                                 __uint_as_float(lop3_and_xor(__float_as_uint(zb), 0x80000000u, wb)));
-            // c + 1/2 from the three exact 0/1 steps, then one fused update of the word
-            const f32x2 s0 = pk2(__saturatef(__fmaf_rn(za, sMa, K0)), __saturatef(__fmaf_rn(zb, sMb, K0)));
-            const f32x2 s1 = pk2(__saturatef(__fmaf_rn(za, sMa, K1)), __saturatef(__fmaf_rn(zb, sMb, K1)));
-            const f32x2 s2 = pk2(__saturatef(__fmaf_rn(za, sMa, K2)), __saturatef(__fmaf_rn(zb, sMb, K2)));
-            W[gg] = fma2(w2, add2(add2(s0, s1), add2(s2, HALF)), W[gg]);
+            const f32x2 w8 = pk2(__uint_as_float((127u + 6u * p) << 23), __uint_as_float((127u + 6u * p + 3u) << 23));
+            const f32x2 x = mul2(pk2(z[2 * i], z[2 * i + 1]), NR);
+            const f32x2 x2 = mul2(x, x);
+            const f32x2 h = fma2(fma2(Q5, x2, Q3), x2, Q1);
+            const f32x2 idx = add2(fma2_rp(h, x, KK), NC);  // 3 + ceil(Q(x))
+            W[gg] = fma2(w8, idx, W[gg]);
         }
     uint32_t g4[4];
 #pragma unroll
@@ -333,32 +332,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float sraw = __fmul_rn(__fdiv_rn(m, nrm), post);
         const float scale = fmaxf(sraw, 1e-8f);
         const float T = (sraw >= 1e-8f) ? m : __fmul_rn(__fmul_rn(1e-8f, nrm), 11.3137085f);
-        const float t0 = __fmul_rn(edge(0), T), t1 = __fmul_rn(edge(1), T), t2 = __fmul_rn(edge(2), T);
-        const uint32_t Mb = (277u - ((__float_as_uint(t0) >> 23) & 0xffu)) << 23;  // 1 / ulp(t0)
-        const float M = __uint_as_float(Mb);
-        const float K0 = -__fmul_rn(t0, M), K1 = -__fmul_rn(t1, M), K2 = -__fmul_rn(t2, M);
+        const float nr = -__frcp_rn(T);
 
-        // pass 2: the indices, 32 columns at a time, the reads alternating as in pass 1
+        // pass 2: the indices, 32 columns at a time. Pieces 2 and 3 are both read before the next
+        // product is released, so that product runs during two pieces' work.
         const int64_t v = (stream + it * n_streams) * kTile + tid;
         int64_t slot = v;  // the slot's load is issued here, ahead of its use at the store
         if constexpr (kLay == tq3::kPool) slot = v < n_vec ? __ldg(static_cast<const int64_t *>(pm.index) + v) : -1;
         uint32_t o[12];
         tmem_wait(za);
         tmem_ld32(my_lanes + 32, zb);
-        bucket_piece(za, Mb, K0, K1, K2, o[0], o[1], o[2]);
+        bucket_piece(za, nr, o[0], o[1], o[2]);
         tmem_wait(zb);
         tmem_ld32(my_lanes + 64, za);
-        bucket_piece(zb, Mb, K0, K1, K2, o[3], o[4], o[5]);
+        bucket_piece(zb, nr, o[3], o[4], o[5]);
         tmem_wait(za);
         tmem_ld32(my_lanes + 96, zb);
-        bucket_piece(za, Mb, K0, K1, K2, o[6], o[7], o[8]);
         tmem_wait(zb);
-        // the accumulator has been read: the next product runs during the last piece's work
+        // the accumulator has been read: the next product runs during the last two pieces' work
         tc_fence_before();
         __syncwarp();
         if ((tid & 31) == 0 && it + 1 < my_tiles && (atom_add_acq_rel(readers, 1u) & 3u) == 3u)
             issue_mma(it + 1);
-        bucket_piece(zb, Mb, K0, K1, K2, o[9], o[10], o[11]);
+        bucket_piece(za, nr, o[6], o[7], o[8]);
+        bucket_piece(zb, nr, o[9], o[10], o[11]);
         if (v < n_vec) {
             if constexpr (kLay != tq3::kSoA) {  // a 56-byte record is 8-byte aligned
                 if (kLay == tq3::kPool && slot >= pm.n_pool) atomicOr(&g_fault, tq3::kFaultPoolIndex);
