@@ -190,6 +190,34 @@ wq_status rpbh_quantize_weight(const void *W, int w_dtype, int64_t rows, int64_t
                                const float *codebook, uint8_t *packed, void *row_norms,
                                void *stream);
 
+/* rpbh_requantize_weight -- OrbitQuantizer.requantize_: the new weight, cast to fp32, is quantized
+ * by _quantize_rows with the module's stored perm, signs and codebook (exactly as
+ * rpbh_quantize_weight), and the row norms are stored in the module's original dtype rather than
+ * the new weight's: row_norms[r] = rho in norm_dtype (WQ_BF16: rounded to nearest even).
+ * rpbh_quantize_weight is this call with norm_dtype = w_dtype.
+ *   row_norms  device, rows entries of norm_dtype, aligned to its size.
+ * Other arguments and errors: as rpbh_quantize_weight (WQ_ERR_DTYPE also for a bad norm_dtype). */
+wq_status rpbh_requantize_weight(const void *W, int w_dtype, int64_t rows, int64_t d,
+                                 const int32_t *perm, const int8_t *signs, int bits,
+                                 const float *codebook, uint8_t *packed, void *row_norms,
+                                 int norm_dtype, void *stream);
+
+/* rpbh_pack_codes / rpbh_unpack_codes -- pack_codes and unpack_codes for any number of codes, on
+ * the device. pack: the low `bits` bits of each of the numel codes go MSB-first into a flat
+ * stream, code k at stream bits bits*k .. bits*k + bits - 1 (stream bit p = bit 7 - p % 8 of byte
+ * p / 8), zero padded to a multiple of 8 codes: ceil(numel / 8) * bits bytes. unpack: the first
+ * numel codes of such a stream, one per byte. A code stream need not start a row on a byte
+ * boundary (the page packs any tensor flat), so this is the form for arrays whose rows hold a
+ * number of codes that is not a multiple of 8; rpbh_quantize_weight writes the same stream for
+ * whole weights.
+ *   codes      device, numel bytes (any alignment; 8-byte aligned is faster).
+ *   packed     device, ceil(numel / 8) * bits bytes (any alignment).
+ *   bits       1 .. 8.
+ * Errors: WQ_ERR_SHAPE (numel < 0 or above 2^46), WQ_ERR_BITS, WQ_ERR_NULL, WQ_ERR_CUDA.
+ * numel == 0 enqueues nothing. */
+wq_status rpbh_pack_codes(const uint8_t *codes, int64_t numel, int bits, uint8_t *packed, void *stream);
+wq_status rpbh_unpack_codes(const uint8_t *packed, int64_t numel, int bits, uint8_t *codes, void *stream);
+
 /* rpbh_dequantize_weight -- _dequantize_rotated, and with unrotate = 1 dequantize.
  * Rotated (unrotate = 0): out[r][j] = codebook[code] * row_norm[r] in out_dtype; for WQ_BF16 the
  * page's bf16 product bf16(bf16(codebook[code]) * bf16(row_norm[r])).

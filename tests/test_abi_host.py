@@ -242,3 +242,29 @@ def test_bindings_reject_buffers_on_another_device_or_dtype(wq):
         wq.rpbh_rotate_activations(torch.zeros(4, 64), perm, signs, out=torch.empty(4, 64, dtype=torch.bfloat16))
     with pytest.raises(ValueError, match="perm must be on"):
         wq.rpbh_rotate_activations(torch.zeros(4, 64), perm.to("meta"), signs)
+
+
+def test_requantize_and_code_packing_argument_validation(wq):
+    """rpbh_requantize_weight checks the norm dtype and its alignment; rpbh_pack_codes and
+    rpbh_unpack_codes check sizes, bits and pointers, all before any device work."""
+    L = wq.lib()
+    WQ_ERR_BITS = -5
+    A = 0x10000
+    cb = np.linspace(-1, 1, 8, dtype=np.float32)
+    rq = lambda w=A, wdt=0, rows=4, d=64, bits=3, norms=A, ndt=1: L.rpbh_requantize_weight(
+        w, wdt, rows, d, A, A, bits, cb.ctypes.data, A, norms, ndt, None)
+    assert rq(rows=0) == WQ_OK
+    assert rq(ndt=7) == WQ_ERR_DTYPE
+    assert rq(wdt=7) == WQ_ERR_DTYPE
+    assert rq(norms=A + 1) == WQ_ERR_ALIGN                          # bf16 norms need 2 bytes
+    assert rq(norms=A + 2, ndt=0) == WQ_ERR_ALIGN                   # fp32 norms need 4 bytes
+    assert rq(norms=None) == WQ_ERR_NULL
+    assert rq(d=40) == WQ_ERR_NOT_QUANTIZABLE
+    assert rq(bits=5) == WQ_ERR_BITS
+    for fn in (L.rpbh_pack_codes, L.rpbh_unpack_codes):
+        assert fn(A, 0, 3, A, None) == WQ_OK
+        assert fn(A, -1, 3, A, None) == WQ_ERR_SHAPE
+        assert fn(A, 8, 0, A, None) == WQ_ERR_BITS
+        assert fn(A, 8, 9, A, None) == WQ_ERR_BITS
+        assert fn(None, 8, 3, A, None) == WQ_ERR_NULL
+        assert fn(A, 8, 3, None, None) == WQ_ERR_NULL

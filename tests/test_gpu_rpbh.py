@@ -207,3 +207,81 @@ def test_misaligned_tables_take_generic_path(wq, oracle):
     x = inputs.activations(rows, d, seed=92)
     out = wq.rpbh_rotate_activations(_t(x, True), pbuf[1:], sbuf[1:])
     assert np.array_equal(_np16(out), oracle.rpbh_rotate_bf16(x, perm, signs, d & -d))
+
+
+# ------------------------------------------------------------------------------------------------
+# requantize_ (norms in the module's original dtype) and pack_codes / unpack_codes on any length
+# ------------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("d,rows", [(96, 37), (3072, 17), (11008, 5), (12288, 2), (6144, 3)])
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("w_bf16,norm_bf16", [(False, True), (True, False), (False, False), (True, True)])
+def test_requantize_norm_dtype(wq, oracle, d, rows, bits, w_bf16, norm_bf16):
+    """Page "orbit_quant.py", requantize_: the new weight in fp32 (or bf16, which casts to fp32
+    exactly) quantized with the stored tables, the norms in the module's original dtype."""
+    w = inputs.gaussian((rows, d), seed=d + rows + bits) * 0.03
+    w[0] *= 50.0
+    if w_bf16:
+        w = inputs.to_bf16_bits(torch.from_numpy(w))
+    perm, signs, perm_d, signs_d = _params(d)
+    cb = oracle.rpbh_codebook(bits, d)
+    ndt = torch.bfloat16 if norm_bf16 else torch.float32
+    packed, norms = wq.rpbh_requantize_weight(_t(w, w_bf16), perm_d, signs_d, bits, cb, ndt)
+    torch.cuda.synchronize()
+    assert norms.dtype == ndt and norms.shape == (rows,)
+    st, ref_packed, ref_norms = parity.check_rpbh_quantize(oracle, w, w_bf16, perm, signs, d & -d, cb, bits,
+                                                            packed.cpu().numpy())
+    if norm_bf16:
+        ref16 = oracle.f32_array_to_bf16(ref_norms).astype(np.int64)
+        assert np.all(np.abs(_np16(norms).astype(np.int64) - ref16) <= 1)
+    else:
+        parity.check_norms(norms.cpu().numpy(), ref_norms)
+    # the same codes as rpbh_quantize_weight, whose norms follow the weight's dtype
+    p2, n2 = wq.rpbh_quantize_weight(_t(w, w_bf16), perm_d, signs_d, bits, cb)
+    assert torch.equal(p2, packed)
+    assert n2.dtype == (torch.bfloat16 if w_bf16 else torch.float32)
+    if n2.dtype == ndt:
+        assert torch.equal(n2, norms)
+
+
+@pytest.mark.parametrize("numel", [1, 5, 7, 8, 9, 63, 1000, 12345, 3 * (1 << 20) + 5])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_pack_unpack_codes_any_length(wq, oracle, numel, bits):
+    """Page "orbit_quant.py", pack_codes / unpack_codes on flat code arrays of any length (a row
+    of 5 or 7 codes starts the next row mid-byte); codes above 2^bits - 1 keep only their low bits,
+    as the page's shifts and masks do. Both directions are compared byte for byte with the oracle."""
+    codes = inputs.uniform_int((numel,), 256, seed=numel * 8 + bits).astype(np.uint8)
+    ref = oracle.pack_codes(codes, bits)
+    got = wq.rpbh_pack_codes(torch.from_numpy(codes).cuda(), bits)
+    assert np.array_equal(got.cpu().numpy(), ref)
+    back = wq.rpbh_unpack_codes(got, bits, numel)
+    assert np.array_equal(back.cpu().numpy(), oracle.unpack_codes(ref, bits, numel))
+    assert np.array_equal(back.cpu().numpy(), codes & ((1 << bits) - 1))
+    # misaligned views (offset by one byte) take the byte-wise path
+    buf = torch.zeros(numel + 1, dtype=torch.uint8, device="cuda")
+    buf[1:] = torch.from_numpy(codes).cuda()
+    got1 = wq.rpbh_pack_codes(buf[1:], bits)
+    assert torch.equal(got1, got)
+    out = torch.zeros(numel + 1, dtype=torch.uint8, device="cuda")
+    wq.rpbh_unpack_codes(got, bits, numel, codes=out[1:])
+    assert torch.equal(out[1:], back) and int(out[0]) == 0
+
+
+def test_pack_codes_of_rows_with_cross_byte_offsets(wq, oracle):
+    """Codes of a [rows, d] array with d not a multiple of 8 (d = 13, 3 bits: 39 bits per row), packed
+    as one stream, then a row read back alone by unpacking the stream and slicing."""
+    rows, d, bits = 77, 13, 3
+    codes = inputs.uniform_int((rows, d), 8, seed=13).astype(np.uint8)
+    got = wq.rpbh_pack_codes(torch.from_numpy(codes).cuda(), bits)
+    assert np.array_equal(got.cpu().numpy(), oracle.pack_codes(codes, bits))
+    back = wq.rpbh_unpack_codes(got, bits, rows * d).view(rows, d)
+    assert np.array_equal(back.cpu().numpy(), codes)
+
+
+def test_pack_codes_errors(wq):
+    from weight_quantization_b200.ops import WQError
+    c = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(WQError):
+        wq.rpbh_pack_codes(c, 9)
+    with pytest.raises(WQError):
+        wq.rpbh_unpack_codes(torch.zeros(16, dtype=torch.uint8, device="cuda"), 0, 16)
+    assert wq.rpbh_pack_codes(c[:0], 3).numel() == 0

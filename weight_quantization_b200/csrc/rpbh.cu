@@ -105,7 +105,7 @@ template <bool kBf16>
 __global__ void __launch_bounds__(kThreads)
     quantize_kernel(const void *__restrict__ w, int d, int h, float post, const int32_t *__restrict__ perm,
                     const int8_t *__restrict__ signs, int bits, Codebook cb, uint8_t *__restrict__ packed,
-                    void *__restrict__ row_norms) {
+                    void *__restrict__ row_norms, int norm_bf16) {
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ double red[33];
     __shared__ float edges[16];
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads)
         for (int b = 0; b < bits; ++b) dst[g * bits + b] = (uint8_t)(word >> (8 * (bits - 1 - b)));
     }
     if (threadIdx.x == 0) {
-        if (kBf16)
+        if (norm_bf16)
             static_cast<uint16_t *>(row_norms)[r] = f32_to_bf16(rho);
         else
             static_cast<float *>(row_norms)[r] = rho;
@@ -278,35 +278,43 @@ extern "C" wq_status rpbh_rotate_activations(const void *x, int dtype, int64_t r
     return launch_status();
 }
 
-extern "C" wq_status rpbh_quantize_weight(const void *W, int w_dtype, int64_t rows, int64_t d, const int32_t *perm,
-                                          const int8_t *signs, int bits, const float *codebook, uint8_t *packed,
-                                          void *row_norms, void *stream) {
+extern "C" wq_status rpbh_requantize_weight(const void *W, int w_dtype, int64_t rows, int64_t d, const int32_t *perm,
+                                            const int8_t *signs, int bits, const float *codebook, uint8_t *packed,
+                                            void *row_norms, int norm_dtype, void *stream) {
     wq_status st = rpbh::check_dims(rows, d);
     if (st != WQ_OK) return st;
     if (bits < 2 || bits > 4) return WQ_ERR_BITS;
-    if (!valid_dtype(w_dtype)) return WQ_ERR_DTYPE;
+    if (!valid_dtype(w_dtype) || !valid_dtype(norm_dtype)) return WQ_ERR_DTYPE;
     if (rows == 0) return WQ_OK;
     if (!W || !perm || !signs || !codebook || !packed || !row_norms) return WQ_ERR_NULL;
-    if (!aligned(W, 16) || !aligned(packed, 4) || !aligned(perm, 4) || !aligned(row_norms, dtype_size(w_dtype)))
+    if (!aligned(W, 16) || !aligned(packed, 4) || !aligned(perm, 4) || !aligned(row_norms, dtype_size(norm_dtype)))
         return WQ_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (rpbh_fast::supported(d, dtype_size(w_dtype), 1) && aligned(perm, 16) && aligned(signs, 16))
-        return rpbh_fast::quantize(W, w_dtype, rows, d, perm, signs, bits, codebook, packed, row_norms, s);
+        return rpbh_fast::quantize(W, w_dtype, rows, d, perm, signs, bits, codebook, packed, row_norms, norm_dtype, s);
     rpbh::Codebook cb = {};
     for (int k = 0; k < (1 << bits); ++k) cb.c[k] = codebook[k];
     const int h = (int)(d & -d);
     const size_t smem = (size_t)d * (4 + dtype_size(w_dtype));
     const float post = rpbh::fwht_post(h);
+    const int nb = norm_dtype == WQ_BF16;
     if (w_dtype == WQ_BF16) {
         if ((st = rpbh::prepare(rpbh::quantize_kernel<true>, smem)) != WQ_OK) return st;
         rpbh::quantize_kernel<true><<<(unsigned)rows, rpbh::kThreads, smem, s>>>(W, (int)d, h, post, perm, signs, bits,
-                                                                                 cb, packed, row_norms);
+                                                                                 cb, packed, row_norms, nb);
     } else {
         if ((st = rpbh::prepare(rpbh::quantize_kernel<false>, smem)) != WQ_OK) return st;
         rpbh::quantize_kernel<false><<<(unsigned)rows, rpbh::kThreads, smem, s>>>(W, (int)d, h, post, perm, signs, bits,
-                                                                                  cb, packed, row_norms);
+                                                                                  cb, packed, row_norms, nb);
     }
     return launch_status();
+}
+
+extern "C" wq_status rpbh_quantize_weight(const void *W, int w_dtype, int64_t rows, int64_t d, const int32_t *perm,
+                                          const int8_t *signs, int bits, const float *codebook, uint8_t *packed,
+                                          void *row_norms, void *stream) {
+    return rpbh_requantize_weight(W, w_dtype, rows, d, perm, signs, bits, codebook, packed, row_norms, w_dtype,
+                                  stream);
 }
 
 namespace {

@@ -193,6 +193,7 @@ struct Edges {
     // steps = 1 when every positive edge is at least 2^-103 (so that M is a normal fp32 value)
     float M[7], K[7];
     int steps;
+    int norm_bf16;  // row norms are stored as bf16 (RNE) when set, fp32 otherwise
 };
 
 __device__ __forceinline__ double block_sum_f64(double v, double *red) {
@@ -392,7 +393,7 @@ __global__ void __launch_bounds__(kMaxThreads)
         for (int k = 0; k < BITS; ++k) reinterpret_cast<uint32_t *>(dst + 4 * BITS * g)[k] = __byte_perm(word[k], 0, 0x0123);
     }
     if (threadIdx.x == 0) {
-        if (kBf16)
+        if (E.norm_bf16)
             static_cast<uint16_t *>(row_norms)[row] = f32_to_bf16(rho);
         else
             static_cast<float *>(row_norms)[row] = rho;
@@ -731,7 +732,7 @@ __global__ void __launch_bounds__(kMaxThreads, 2)
                 reinterpret_cast<uint32_t *>(dst + 4 * BITS * g)[k] = __byte_perm(word[k], 0, 0x0123);
         }
         if (threadIdx.x == 0) {
-            if (kBf16)
+            if (E.norm_bf16)
                 static_cast<uint16_t *>(row_norms)[row] = f32_to_bf16(rho);
             else
                 static_cast<float *>(row_norms)[row] = rho;
@@ -891,7 +892,7 @@ __global__ void __launch_bounds__(kSlotsT == 1 ? 128 : kMaxThreads, kSlotsT == 1
         }
         __syncwarp();  // the codes are read before the next row's pass 0 rewrites this part of the buffer
         if (threadIdx.x == 0) {
-            if (kBf16)
+            if (E.norm_bf16)
                 static_cast<uint16_t *>(row_norms)[row] = f32_to_bf16(rho);
             else
                 static_cast<float *>(row_norms)[row] = rho;
@@ -1333,9 +1334,10 @@ wq_status quantize_sym(bool bf, bool sym, int bits, const void *w, int64_t rows,
 }
 
 wq_status quantize(const void *w, int w_dtype, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
-                   int bits, const float *codebook, uint8_t *packed, void *row_norms, cudaStream_t s) {
+                   int bits, const float *codebook, uint8_t *packed, void *row_norms, int norm_dtype, cudaStream_t s) {
     const int L = 1 << bits;
     Edges E = {};
+    E.norm_bf16 = norm_dtype == WQ_BF16;
     // edges = (codebook[:-1] + codebook[1:]) / 2, in fp32 as the page computes them
     for (int k = 0; k + 1 < L; ++k) {
         volatile float sum = codebook[k] + codebook[k + 1];

@@ -17,8 +17,9 @@ bool supported(int64_t d, int in_esz, int out_esz);
 wq_status rotate(const void *x, int dtype, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
                  void *out, cudaStream_t s);
 
+// Row norms are written in norm_dtype (WQ_F32 or WQ_BF16), whatever the weight's dtype.
 wq_status quantize(const void *w, int w_dtype, int64_t rows, int64_t d, const int32_t *perm, const int8_t *signs,
-                   int bits, const float *codebook, uint8_t *packed, void *row_norms, cudaStream_t s);
+                   int bits, const float *codebook, uint8_t *packed, void *row_norms, int norm_dtype, cudaStream_t s);
 
 wq_status dequantize_unrotate(const uint8_t *packed, const void *row_norms, int norm_dtype, int64_t rows, int64_t d,
                               int bits, const float *codebook, const int32_t *perm, const int8_t *signs, void *out,

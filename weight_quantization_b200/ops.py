@@ -32,6 +32,9 @@ PROTOTYPES = {
     "tq3_attention": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _vp, C.c_float, _vp, _int, _vp]),
     "tq3_compressed_bytes": (_i64, [_i64]),
     "rpbh_quantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp]),
+    "rpbh_requantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _int, _vp]),
+    "rpbh_pack_codes": (_int, [_vp, _i64, _int, _vp, _vp]),
+    "rpbh_unpack_codes": (_int, [_vp, _i64, _int, _vp, _vp]),
     "rpbh_dequantize_weight": (_int, [_vp, _vp, _int, _i64, _i64, _int, _vp, _vp, _vp, _int, _vp, _int, _vp]),
     "rpbh_rotate_activations": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _vp, _vp]),
     "rpbh_linear": (_int, [_vp, _vp, _int, _i64, _i64, _int, _vp, _vp, _i64, _vp, _vp, _vp]),
@@ -315,6 +318,62 @@ def rpbh_quantize_weight(W: torch.Tensor, perm: torch.Tensor, signs: torch.Tenso
                                     _dev(row_norms, "row_norms"), _stream(W.device))
     _check("rpbh_quantize_weight", st)
     return packed, row_norms
+
+
+def rpbh_requantize_weight(W: torch.Tensor, perm: torch.Tensor, signs: torch.Tensor, bits: int, codebook,
+                           norm_dtype, packed=None, row_norms=None):
+    """requantize_: quantize W [rows, d] (fp32/bf16) with the stored perm, signs and codebook, the
+    row norms in norm_dtype (the module's original dtype). Returns (packed, row_norms)."""
+    rows, d = W.shape
+    cb = _codebook_arg(codebook, bits)
+    if norm_dtype not in _DT:
+        raise ValueError("norm_dtype must be torch.float32 or torch.bfloat16")
+    if packed is None:
+        packed = torch.empty(max(rpbh_packed_bytes(rows, d, bits), 0), dtype=torch.uint8, device=W.device)
+    if row_norms is None:
+        row_norms = torch.empty(rows, dtype=norm_dtype, device=W.device)
+    for name, t in (("packed", packed), ("perm", perm), ("signs", signs)):
+        _on(t, W.device, name)
+    _on(row_norms, W.device, "row_norms", (norm_dtype,))
+    _fits(packed, rpbh_packed_bytes(rows, d, bits), "packed")
+    _fits(row_norms, rows, "row_norms")
+    _fits(perm, d, "perm")
+    _fits(signs, d, "signs")
+    st = lib().rpbh_requantize_weight(_dev(W, "W"), _DT.get(W.dtype, -1), rows, d, _dev(perm, "perm"),
+                                      _dev(signs, "signs"), bits, cb.ctypes.data, _dev(packed, "packed"),
+                                      _dev(row_norms, "row_norms"), _DT[norm_dtype], _stream(W.device))
+    _check("rpbh_requantize_weight", st)
+    return packed, row_norms
+
+
+def rpbh_pack_codes(codes: torch.Tensor, bits: int, packed=None):
+    """pack_codes: codes (uint8, any shape, flattened) -> flat MSB-first stream of
+    ceil(numel / 8) * bits bytes."""
+    if codes.dtype != torch.uint8:
+        raise ValueError("codes must be uint8")
+    numel = codes.numel()
+    nbytes = (numel + 7) // 8 * bits
+    if packed is None:
+        packed = torch.empty(nbytes, dtype=torch.uint8, device=codes.device)
+    _on(packed, codes.device, "packed", (torch.uint8,))
+    _fits(packed, nbytes, "packed")
+    st = lib().rpbh_pack_codes(_dev(codes, "codes"), numel, bits, _dev(packed, "packed"), _stream(codes.device))
+    _check("rpbh_pack_codes", st)
+    return packed
+
+
+def rpbh_unpack_codes(packed: torch.Tensor, bits: int, numel: int, codes=None):
+    """unpack_codes: the first numel codes of a packed stream, as uint8 [numel]."""
+    if packed.dtype != torch.uint8:
+        raise ValueError("packed must be uint8")
+    _fits(packed, (numel + 7) // 8 * bits, "packed")
+    if codes is None:
+        codes = torch.empty(numel, dtype=torch.uint8, device=packed.device)
+    _on(codes, packed.device, "codes", (torch.uint8,))
+    _fits(codes, numel, "codes")
+    st = lib().rpbh_unpack_codes(_dev(packed, "packed"), numel, bits, _dev(codes, "codes"), _stream(packed.device))
+    _check("rpbh_unpack_codes", st)
+    return codes
 
 
 def rpbh_dequantize_weight(packed: torch.Tensor, row_norms: torch.Tensor, rows: int, d: int, bits: int, codebook,
