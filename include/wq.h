@@ -140,7 +140,7 @@ wq_status tq3_decode_paged(const uint8_t *pool, int64_t n_pool, const int32_t *p
  * No mask: every row attends to all S keys of its head.
  *   q          device, heads x m x 128 elements of q_dtype. The m rows of a head share its keys and
  *              values (grouped-query attention: m = query heads per KV head x query tokens).
- *   m          1 .. 16.
+ *   m          1 .. 2^20 (rows are served 16 at a time; each group of 16 reads the records again).
  *   k_records, v_records  device, heads x S x 56 bytes (the tq3_encode_aos record), 8-byte aligned.
  *   S          1 .. 2^31 keys per head.
  *   softmax_scale  finite; 1/sqrt(128) is the usual value. (Any finite fp32 scale keeps the
@@ -156,6 +156,21 @@ wq_status tq3_decode_paged(const uint8_t *pool, int64_t n_pool, const int32_t *p
 wq_status tq3_attention(const void *q, int q_dtype, int64_t heads, int64_t m, const uint8_t *k_records,
                         const uint8_t *v_records, int64_t S, const uint32_t *sign_mask, float softmax_scale,
                         void *out, int out_dtype, void *stream);
+
+/* tq3_attention_paged -- tq3_attention with the keys and values read from a paged cache: pools of
+ * 56-byte records (as tq3_encode_slots writes them) shared by all heads, and a page table. Key j of
+ * head h is record page_table[h * pages_per_head + j / page_size] * page_size + j % page_size of
+ * k_pool and of v_pool (a K page and its V page share the entry).
+ *   k_pool, v_pool  device, n_pool x 56 bytes each, 8-byte aligned.
+ *   page_table device, heads x pages_per_head int32, 4-byte aligned; S <= pages_per_head * page_size.
+ *   page_size  a power of two, 1 .. 2^30.
+ * A page-table entry that is negative or names records at or beyond n_pool masks those keys out
+ * (weight 0) and sets device fault bit 6; a head whose keys are all masked gives NaN rows.
+ * Other arguments, precision and errors: as tq3_attention. */
+wq_status tq3_attention_paged(const void *q, int q_dtype, int64_t heads, int64_t m, const uint8_t *k_pool,
+                              const uint8_t *v_pool, int64_t n_pool, const int32_t *page_table,
+                              int64_t pages_per_head, int64_t page_size, int64_t S, const uint32_t *sign_mask,
+                              float softmax_scale, void *out, int out_dtype, void *stream);
 
 /* tq3_compressed_bytes -- tq3_memory_bytes' compressed size for n_vec vectors: 56 * n_vec
  * (-1 if n_vec < 0 or the product overflows). */
@@ -288,9 +303,9 @@ wq_status wq_rpbh_codebook(int bits, int64_t d, float *out);
  * leaving its outputs unspecified: bit 0 a TQ3 kernel waiting for a TMA tile, bit 1 an RPBH kernel
  * waiting for a row copy, bit 3 the tensor-core TQ3 encoder waiting for a tile or its product,
  * bit 4 rpbh_linear waiting for a tile, the unpacked weights or its product, bit 5 the self-test
- * wq_selftest_wait_timeout. Bit 6 is not a wait: tq3_encode_slots or tq3_decode_paged met a slot or
- * page-table entry outside the pool (that record was skipped, or decoded as zeros; the rest of the
- * call is complete).
+ * wq_selftest_wait_timeout. Bit 6 is not a wait: tq3_encode_slots, tq3_decode_paged or
+ * tq3_attention_paged met a slot or page-table entry outside the pool (that record was skipped,
+ * decoded as zeros, or masked out of the attention; the rest of the call is complete).
  * Synchronous (a device-to-host copy on the legacy default stream); `flags` is host memory.
  * Errors: WQ_ERR_NULL, WQ_ERR_CUDA. */
 wq_status wq_device_fault(unsigned int *flags);

@@ -167,7 +167,7 @@ def test_record_pool_and_attention_argument_validation(wq):
     attn = lambda q=A, qdt=1, heads=2, rows=4, k=A, v=A, S=100, scale=0.088, out=A, odt=1: \
         L.tq3_attention(q, qdt, heads, rows, k, v, S, mp, scale, out, odt, None)
     assert attn(heads=0) == WQ_OK
-    for rows in (0, 17):
+    for rows in (0, (1 << 20) + 1):                                       # 1 .. 2^20 rows (chunks of 16)
         assert attn(rows=rows) == WQ_ERR_SHAPE
     for S in (0, (1 << 31) + 1):
         assert attn(S=S) == WQ_ERR_SHAPE
@@ -179,6 +179,19 @@ def test_record_pool_and_attention_argument_validation(wq):
     assert attn(k=A + 4) == WQ_ERR_ALIGN
     assert attn(q=A + 1) == WQ_ERR_ALIGN                                   # bf16 needs 2 bytes
     assert attn(out=A + 2, odt=0) == WQ_ERR_ALIGN                          # fp32 needs 4 bytes
+
+    pa = lambda q=A, heads=2, rows=4, k=A, v=A, n_pool=64, tab=A, pph=4, ps=16, S=60, scale=0.088, out=A: \
+        L.tq3_attention_paged(q, 1, heads, rows, k, v, n_pool, tab, pph, ps, S, mp, scale, out, 1, None)
+    assert pa(heads=0) == WQ_OK
+    assert pa(S=65) == WQ_ERR_SHAPE                                        # more than the table covers
+    for ps in (0, 12, 1 << 31):
+        assert pa(ps=ps) == WQ_ERR_SHAPE
+    assert pa(n_pool=-1) == WQ_ERR_SHAPE
+    assert pa(pph=-1) == WQ_ERR_SHAPE
+    assert pa(scale=float("nan")) == WQ_ERR_SHAPE
+    assert pa(tab=None) == WQ_ERR_NULL
+    assert pa(tab=A + 2) == WQ_ERR_ALIGN
+    assert pa(k=A + 4) == WQ_ERR_ALIGN
 
 
 def test_bindings_reject_buffers_smaller_than_the_call(wq):

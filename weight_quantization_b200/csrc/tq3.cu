@@ -429,6 +429,10 @@ extern "C" wq_status wq_selftest_wait_timeout(void *stream) {
     return launch_status();
 }
 
+namespace wq {
+unsigned int tq3_attn_read_and_clear_fault();  // tq3_attn.cu
+}
+
 extern "C" wq_status wq_device_fault(unsigned int *flags) {
     if (!flags) return WQ_ERR_NULL;
     unsigned int v = 0, zero = 0;
@@ -438,7 +442,8 @@ extern "C" wq_status wq_device_fault(unsigned int *flags) {
     const unsigned int q = tq3_rows::read_and_clear_fault();
     const unsigned int t = tq3_mma::read_and_clear_fault();
     const unsigned int l = rpbh_linear::read_and_clear_fault();
-    if ((r | q | t | l) & 0x80000000u) return WQ_ERR_CUDA;
-    *flags = v | r | q | t | l;
+    const unsigned int a = tq3_attn_read_and_clear_fault();
+    if ((r | q | t | l | a) & 0x80000000u) return WQ_ERR_CUDA;
+    *flags = v | r | q | t | l | a;
     return WQ_OK;
 }

@@ -30,6 +30,8 @@ PROTOTYPES = {
     "tq3_encode_slots": (_int, [_vp, _int, _i64, _vp, _vp, _vp, _i64, _vp]),
     "tq3_decode_paged": (_int, [_vp, _i64, _vp, _i64, _i64, _i64, _vp, _vp, _int, _vp]),
     "tq3_attention": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _vp, C.c_float, _vp, _int, _vp]),
+    "tq3_attention_paged": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _i64, _vp, _i64, _i64, _i64, _vp, C.c_float,
+                                   _vp, _int, _vp]),
     "tq3_compressed_bytes": (_i64, [_i64]),
     "rpbh_quantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _vp]),
     "rpbh_requantize_weight": (_int, [_vp, _int, _i64, _i64, _vp, _vp, _int, _vp, _vp, _vp, _int, _vp]),
@@ -277,6 +279,37 @@ def tq3_attention(q: torch.Tensor, k_records: torch.Tensor, v_records: torch.Ten
                              _dev(v_records, "v_records"), k_records.shape[1], msk.ctypes.data,
                              float(softmax_scale), _dev(out, "out"), _DT[out.dtype], _stream(q.device))
     _check("tq3_attention", st)
+    return out
+
+
+def tq3_attention_paged(q: torch.Tensor, k_pool: torch.Tensor, v_pool: torch.Tensor, page_table: torch.Tensor,
+                        page_size: int, S: int, sign_mask, softmax_scale: float = 128 ** -0.5, out_dtype=None,
+                        out=None):
+    """tq3_attention over a paged cache: q [heads, m, 128]; k_pool, v_pool [n_pool, 56] records;
+    page_table int32 [heads, pages_per_head]; key j of head h is record
+    page_table[h, j // page_size] * page_size + j % page_size. Returns [heads, m, 128]."""
+    if q.dtype not in _DT or q.ndim != 3 or q.shape[2] != 128:
+        raise ValueError("q must be [heads, m, 128] float32 or bfloat16")
+    heads, m = q.shape[0], q.shape[1]
+    for name, t in (("k_pool", k_pool), ("v_pool", v_pool)):
+        if t.dtype != torch.uint8 or t.ndim != 2 or t.shape[1] != 56:
+            raise ValueError(f"{name} must be uint8 [n_pool, 56]")
+    if k_pool.shape != v_pool.shape:
+        raise ValueError("k_pool and v_pool must have the same shape")
+    if page_table.dtype != torch.int32 or page_table.ndim != 2 or page_table.shape[0] != heads:
+        raise ValueError("page_table must be int32 [heads, pages_per_head]")
+    if out is None:
+        out = torch.empty((heads, m, 128), dtype=out_dtype or q.dtype, device=q.device)
+    for name, t in (("k_pool", k_pool), ("v_pool", v_pool), ("page_table", page_table)):
+        _on(t, q.device, name)
+    _on(out, q.device, "out", _DT)
+    _fits(out, heads * m * 128, "out")
+    msk = _mask_arg(sign_mask)
+    st = lib().tq3_attention_paged(_dev(q, "q"), _DT[q.dtype], heads, m, _dev(k_pool, "k_pool"),
+                                   _dev(v_pool, "v_pool"), k_pool.shape[0], _dev(page_table, "page_table"),
+                                   page_table.shape[1], int(page_size), int(S), msk.ctypes.data, float(softmax_scale),
+                                   _dev(out, "out"), _DT[out.dtype], _stream(q.device))
+    _check("tq3_attention_paged", st)
     return out
 
 
