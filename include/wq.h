@@ -149,8 +149,12 @@ wq_status tq3_decode_paged(const uint8_t *pool, int64_t n_pool, const int32_t *p
  *              overflows makes the head's output undefined, as NaN or Inf inputs do.
  *   out        device, heads x m x 128 elements of out_dtype (bf16: rounded once, to nearest even).
  * Precision: the keys and values are never decoded; the query is rotated once into the basis the
- * indices live in and the output rotated back once, in fp32. The result differs from attention over
- * the decoded fp32 vectors by fp32 rounding only.
+ * indices live in and the output rotated back once, in fp32. Below 48 rows per head the products run
+ * on the CUDA cores in fp32 and the result differs from attention over the decoded fp32 vectors by
+ * fp32 rounding only. From 48 rows on they run on the tensor cores (tcgen05, 128 rows per CTA) on
+ * bf16 operands, each fp32 operand split into hi + lo and three passes accumulated in fp32: a logit
+ * is then within about 2^-14 softmax_scale |q| |k| of its fp32 value and a value sum within
+ * (3 * 2^-18 + (432 + S / 128) 2^-24) max|v| per element.
  * Errors: WQ_ERR_SHAPE (heads < 0, m or S out of range, softmax_scale not finite), WQ_ERR_DTYPE,
  * WQ_ERR_NULL, WQ_ERR_ALIGN (q and out to their element size). heads == 0 enqueues nothing. */
 wq_status tq3_attention(const void *q, int q_dtype, int64_t heads, int64_t m, const uint8_t *k_records,
@@ -303,7 +307,7 @@ wq_status wq_rpbh_codebook(int bits, int64_t d, float *out);
  * leaving its outputs unspecified: bit 0 a TQ3 kernel waiting for a TMA tile, bit 1 an RPBH kernel
  * waiting for a row copy, bit 3 the tensor-core TQ3 encoder waiting for a tile or its product,
  * bit 4 rpbh_linear waiting for a tile, the unpacked weights or its product, bit 5 the self-test
- * wq_selftest_wait_timeout. Bit 6 is not a wait: tq3_encode_slots, tq3_decode_paged or
+ * wq_selftest_wait_timeout, bit 7 the tensor-core attention waiting for its product. Bit 6 is not a wait: tq3_encode_slots, tq3_decode_paged or
  * tq3_attention_paged met a slot or page-table entry outside the pool (that record was skipped,
  * decoded as zeros, or masked out of the attention; the rest of the call is complete).
  * Synchronous (a device-to-host copy on the legacy default stream); `flags` is host memory.

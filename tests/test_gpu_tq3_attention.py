@@ -19,7 +19,20 @@ Tolerance, from the arithmetic (u = 2^-24, first order):
   added, n = ceil(S / splits) + ceil(S / 128) + 8. The inverse transform adds seven stages; bounded
   as above this is (n + 40) u max_j |v_j|_2 on every output element.
 * bf16 output: one rounding, 2^-8 |out| allowed.
+
+From 48 query rows per head on, the call takes the tensor-core path: the products run on bf16
+operands, each fp32 operand split into hi + lo (residual at most 2^-18 of the value) and three
+passes hi hi + hi lo + lo hi accumulated in fp32. Per product term that adds 3 * 2^-18 (two split
+residuals and the dropped lo lo) and one rounding of the folded key or value factor, and each
+128-key tile accumulates 3 * 128 = 384 terms; so there
+* logits: |d logit_j| <= (3 * 2^-18 + (384 + 7 sqrt(128) + 12) u) softmax_scale |q| |k_j|, below
+  2^-14 softmax_scale |q| max_j |k_j| =: L_tc, and the weights move as above with L_tc for L;
+* values: (3 * 2^-18 + (384 + ceil(S / 128) + 48) u) max_j |v_j|_2 on every output element (the
+  tile products, the per-tile accumulation in tensor memory and the rare rescales of the running
+  max).
 """
+
+MMA_MIN_ROWS = 48
 import math
 
 import numpy as np
@@ -55,13 +68,20 @@ def _cache(oracle, heads, S, seed):
 
 
 def _tolerance(qf, k, v, S, scale, ref, out_bf16):
-    splits = min(8, -(-S // 256))
-    n = -(-S // splits) + -(-S // 128) + 8
+    m = qf.shape[1]
     vinf = np.abs(v).max(axis=(1, 2))                   # per head
     v2 = np.linalg.norm(v, axis=2).max(axis=1)
     k2 = np.linalg.norm(k, axis=2).max(axis=1)
-    L = 2.0 ** -16 * scale * np.linalg.norm(qf.astype(np.float64), axis=2) * k2[:, None]   # [heads, m]
-    tol = (4.4 * L + 2.0 ** -21)[:, :, None] * vinf[:, None, None] + ((n + 40) * U * v2)[:, None, None]
+    qn = np.linalg.norm(qf.astype(np.float64), axis=2)
+    if m >= MMA_MIN_ROWS:                               # tensor-core path
+        L = 2.0 ** -14 * scale * qn * k2[:, None]
+        eps = 3 * 2.0 ** -18 + (384 + -(-S // 128) + 48) * U
+    else:
+        splits = min(8, -(-S // 256))
+        n = -(-S // splits) + -(-S // 128) + 8
+        L = 2.0 ** -16 * scale * qn * k2[:, None]      # [heads, m]
+        eps = (n + 40) * U
+    tol = (4.4 * L + 2.0 ** -21)[:, :, None] * vinf[:, None, None] + (eps * v2)[:, None, None]
     if out_bf16:
         tol = tol + 2.0 ** -8 * np.abs(ref)
     return tol
@@ -92,7 +112,8 @@ def _check(wq, oracle, heads, m, S, q_bf16, out_bf16, scale, seed):
 
 
 @pytest.mark.parametrize("heads,m,S", [(1, 1, 1), (3, 4, 127), (2, 8, 1000), (5, 16, 4097), (2, 3, 128 * 8 * 3 + 5),
-                                       (4, 2, 129), (2, 17, 700), (2, 32, 2049), (1, 128, 1500), (3, 40, 256)])
+                                       (4, 2, 129), (2, 17, 700), (2, 32, 2049), (1, 128, 1500), (3, 40, 256),
+                                       (2, 48, 129), (3, 64, 1000), (2, 130, 300), (1, 256, 4096)])
 @pytest.mark.parametrize("q_bf16", [True, False])
 def test_attention_matches_oracle(wq, oracle, heads, m, S, q_bf16):
     _check(wq, oracle, heads, m, S, q_bf16, False, 128 ** -0.5, seed=heads * 1000 + m * 10 + S)
@@ -120,7 +141,8 @@ def test_attention_argument_errors(wq):
     assert wq.tq3_attention(torch.zeros(0, 1, 128, device="cuda"), rec[:0], rec[:0], mask).shape == (0, 1, 128)
 
 
-@pytest.mark.parametrize("heads,m,S,page_size", [(3, 4, 1000, 16), (2, 8, 4097, 128), (2, 1, 300, 1), (1, 20, 777, 64)])
+@pytest.mark.parametrize("heads,m,S,page_size", [(3, 4, 1000, 16), (2, 8, 4097, 128), (2, 1, 300, 1), (1, 20, 777, 64),
+                                                  (2, 128, 1000, 32)])
 def test_attention_paged_matches_oracle(wq, oracle, heads, m, S, page_size):
     """tq3_attention_paged: the heads' pages scattered in random order over a pool (with unused
     records between them), against the oracle on the records gathered back into order."""

@@ -38,6 +38,7 @@
 #include <string.h>
 
 #include "common.cuh"
+#include "tq3_attn_mma.cuh"
 #include "tq3_common.cuh"
 #include "wq.h"
 
@@ -56,14 +57,10 @@ constexpr int kThreads = 128;
 
 __device__ unsigned int g_fault;
 
-// Where the records of (head, key) live: contiguous [heads][S] records, or a pool reached through a
-// page table of pages_per_head int32 entries per head.
-struct KV {
-    const uint8_t *k, *v;
-    const int32_t *table;  // null: contiguous
-    int64_t pages_per_head, n_pool;
-    int shift;             // log2 of the page size
-};
+using KV = AttnCache;
+
+// From this many query rows per head on, the tensor-core kernel (tq3_attn_mma.cu) serves the call.
+constexpr int64_t kMmaMinRows = 48;
 
 // Record index of key j of head h, or -1 for a page-table entry outside the pool.
 __device__ __forceinline__ int64_t record_of(const KV &kv, int64_t head, int64_t S, int64_t j) {
@@ -462,6 +459,7 @@ wq_status launch(const void *q, int q_dtype, int64_t heads, int m, int m_total, 
 // Every chunk of up to kMaxRows query rows of every head, one launch per chunk.
 wq_status run(const void *q, int q_dtype, int64_t heads, int64_t m, const KV &kv, int64_t S, const SignMask &mask,
               float coef, void *out, int out_dtype, cudaStream_t s) {
+    if (m >= kMmaMinRows) return tq3_attn_mma::run(q, q_dtype, heads, m, kv, S, mask, coef, out, out_dtype, s);
     for (int64_t r0 = 0; r0 < m; r0 += kMaxRows) {
         const int mc = (int)(m - r0 < kMaxRows ? m - r0 : kMaxRows);
         wq_status st;
@@ -495,7 +493,7 @@ unsigned int tq3_attn_read_and_clear_fault() {
     unsigned int v = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&v, tq3_attn::g_fault, sizeof v) != cudaSuccess) return 0x80000000u;
     if (v) cudaMemcpyToSymbol(tq3_attn::g_fault, &zero, sizeof zero);
-    return v;
+    return v | tq3_attn_mma::read_and_clear_fault();
 }
 
 }  // namespace wq
