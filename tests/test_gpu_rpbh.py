@@ -51,7 +51,8 @@ def _quantize_and_check(wq, oracle, w, is_bf16, d, bits):
 
 
 @pytest.mark.parametrize("d,rows", [(32, 5), (96, 37), (192, 11), (256, 3), (1024, 9), (3072, 17), (640, 1),
-                                    (4096, 3), (12288, 2), (6400, 7), (9472, 5), (1536, 3), (6144, 2)])
+                                    (4096, 3), (12288, 2), (6400, 7), (9472, 5), (1536, 3), (6144, 2), (768, 4),
+                                    (13056, 1), (13056, 3), (15360, 2)])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 @pytest.mark.parametrize("is_bf16", [False, True])
 def test_quantize_small(wq, oracle, d, rows, bits, is_bf16):
@@ -139,7 +140,8 @@ def test_quantize_then_dequantize_llm_roundtrip(wq, oracle):
 
 
 @pytest.mark.parametrize("rows,d", [(2048, 11008), (4096, 3072), (3, 96), (1, 32), (5, 192), (3, 4096),
-                                    (7, 640), (9, 2880), (5, 6400), (3, 1536), (2, 6144)])
+                                    (7, 640), (9, 2880), (5, 6400), (3, 1536), (2, 6144), (3, 256), (4, 768),
+                                    (2, 1024), (5, 13056), (3, 15360), (301, 3072)])
 def test_rotate_activations(wq, oracle, rows, d):
     perm, signs, perm_d, signs_d = _params(d)
     h = d & -d

@@ -43,10 +43,16 @@ def build(force: bool = False, verbose: bool = False) -> str:
               "-I", os.path.join(ROOT, "include"), "-I", os.path.join(PKG, "csrc")] + ARCH
     if verbose:
         common += ["-Xptxas", "-v"]
+    # an object is reused when it is newer than its source and every header (and this script)
+    headers = [h for h in _deps() if not h.endswith((".cu", ".cpp"))] + [os.path.abspath(__file__)]
+    newest_header = max(os.path.getmtime(h) for h in headers)
     objs = []
     for src in sources():
         obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
-        subprocess.run([NVCC, "-c", src, "-o", obj] + common, check=True)
+        fresh = (not force and os.path.exists(obj) and
+                 os.path.getmtime(obj) > max(os.path.getmtime(src), newest_header))
+        if not fresh:
+            subprocess.run([NVCC, "-c", src, "-o", obj] + common, check=True)
         objs.append(obj)
     tmp = LIB + ".tmp"
     subprocess.run([NVCC, "-shared", "-o", tmp] + objs + ARCH + ["-cudart", "static", "-Xlinker", "--no-undefined"],

@@ -431,6 +431,9 @@ extern "C" wq_status wq_selftest_wait_timeout(void *stream) {
 
 namespace wq {
 unsigned int tq3_attn_read_and_clear_fault();  // tq3_attn.cu
+namespace rpbh_lanes {
+unsigned int read_and_clear_fault();  // rpbh_lanes.cu
+}
 }
 
 extern "C" wq_status wq_device_fault(unsigned int *flags) {
@@ -443,7 +446,8 @@ extern "C" wq_status wq_device_fault(unsigned int *flags) {
     const unsigned int t = tq3_mma::read_and_clear_fault();
     const unsigned int l = rpbh_linear::read_and_clear_fault();
     const unsigned int a = tq3_attn_read_and_clear_fault();
-    if ((r | q | t | l | a) & 0x80000000u) return WQ_ERR_CUDA;
-    *flags = v | r | q | t | l | a;
+    const unsigned int n = rpbh_lanes::read_and_clear_fault();
+    if ((r | q | t | l | a | n) & 0x80000000u) return WQ_ERR_CUDA;
+    *flags = v | r | q | t | l | a | n;
     return WQ_OK;
 }
