@@ -124,7 +124,7 @@ def traffic_bytes(kernel: str):
     if not os.path.exists(p):
         return None
     src = {"tq3_encode": "tq3_mma.cu", "tq3_decode": "tq3_rows.cu", "tq3_encode_exact": "tq3.cu",
-           "rpbh_quantize": "rpbh_fast.cu", "rpbh_rotate": "rpbh_fast.cu", "rpbh_dequantize": "rpbh_fast.cu",
+           "rpbh_quantize": "rpbh_lanes.cu", "rpbh_rotate": "rpbh_lanes.cu", "rpbh_dequantize": "rpbh_fast.cu",
            "rpbh_linear": "rpbh_linear.cu", "tq3_attention": "tq3_attn.cu"}.get(kernel)
     if src is None:
         return None

@@ -24,8 +24,8 @@ def test_peaks_come_from_the_measured_file():
 
 def test_traffic_is_reported_only_for_the_source_it_was_taken_on():
     import bench
-    src = {"tq3_encode": "tq3_mma.cu", "tq3_decode": "tq3_rows.cu", "rpbh_quantize": "rpbh_fast.cu",
-           "rpbh_linear": "rpbh_linear.cu", "tq3_attention": "tq3_attn.cu"}
+    src = {"tq3_encode": "tq3_mma.cu", "tq3_decode": "tq3_rows.cu", "rpbh_quantize": "rpbh_lanes.cu",
+           "rpbh_rotate": "rpbh_lanes.cu", "rpbh_linear": "rpbh_linear.cu", "tq3_attention": "tq3_attn.cu"}
     lines = [l.split() for l in open(os.path.join(ROOT, "profiles", "traffic.txt")) if l.strip() and not l.startswith("#")]
     assert lines
     for name, sha, _, value in lines:
