@@ -213,10 +213,34 @@ struct Xpose {
     }
 };
 
-// 32 codes (code i in byte i of cw) to BITS words of the MSB-first stream.
+// 3-bit decisions as rpbh_fast::sym_codes, with the sign applied by one packed fma:
+// 2^22 + mid + 1/2 + sgn (c + 1/2), exact, whose low byte is twice the code.
+__device__ __forceinline__ f32x2 sym_codes3x2(f32x2 u, const Edges &E) {
+    float u0, u1;
+    upk2(u, u0, u1);
+    const f32x2 ap = rpbh_fast::fma_rp2(u, pk2(-0x1p-24f, -0x1p-24f), pk2(fabsf(u0), fabsf(u1)));
+    float a0, a1;
+    upk2(ap, a0, a1);
+    f32x2 c = pk2(0.5f, 0.5f);
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+        c = add2(c, pk2(__saturatef(__fmaf_rn(a0, E.M[i], E.K[i])), __saturatef(__fmaf_rn(a1, E.M[i], E.K[i]))));
+    float b0, b1;
+    upk2(rpbh_fast::fma_rm2(u, pk2(1.0f, 1.0f), pk2(-0.0f, -0.0f)), b0, b1);
+    const f32x2 sg = pk2(__uint_as_float((__float_as_uint(b0) & 0x80000000u) | 0x3f800000u),
+                         __uint_as_float((__float_as_uint(b1) & 0x80000000u) | 0x3f800000u));
+    constexpr float kB = 4194304.0f + 3.5f;  // 2^22 + mid + 1/2
+    return fma2(sg, c, pk2(kB, kB));
+}
+
+// 32 codes to BITS words of the MSB-first stream: code i in byte i of cw (3 bits: twice the code,
+// as sym_codes3x2 leaves it).
 template <int BITS>
 __device__ __forceinline__ void pack_unit(const uint32_t (&cw)[8], uint32_t (&word)[BITS]) {
     if constexpr (BITS == 3) {
+        // each word of four bytes (twice the codes c0 .. c3) gives twice the 12-bit chunk
+        // c0 c1 c2 c3 (MSB first) by two 16x8-bit dot products (weights 512, 64 on bytes 0, 1, then
+        // 8, 1 on bytes 2, 3); the shifts below halve it while placing the eight chunks
         uint32_t ch[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -224,12 +248,12 @@ __device__ __forceinline__ void pack_unit(const uint32_t (&cw)[8], uint32_t (&wo
             asm("dp2a.lo.u32.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(0x00400200u), "r"(cw[j]), "r"(0u));
             asm("dp2a.hi.u32.u32 %0, %1, %2, %3;" : "=r"(ch[j]) : "r"(0x00010008u), "r"(cw[j]), "r"(r));
         }
-        word[0] = (ch[0] << 20) | (ch[1] << 8) | (ch[2] >> 4);
-        word[1] = (ch[2] << 28) | (ch[3] << 16) | (ch[4] << 4) | (ch[5] >> 8);
-        word[2] = (ch[5] << 24) | (ch[6] << 12) | ch[7];
-    }
-    else
+        word[0] = (ch[0] << 19) | (ch[1] << 7) | (ch[2] >> 5);
+        word[1] = (ch[2] << 27) | (ch[3] << 15) | (ch[4] << 3) | (ch[5] >> 9);
+        word[2] = (ch[5] << 23) | (ch[6] << 11) | (ch[7] >> 1);
+    } else {
         rpbh_fast::pack32<BITS>(cw, word);
+    }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -375,7 +399,10 @@ __global__ void __maxnreg__(B == 4 ? 80 : 96)
                     const f32x2 q0 = mul2(z, RDEN);
                     const f32x2 u = fma2(fma2(q0, NDEN, z), RDEN, q0);
                     float v0, v1;
-                    upk2(rpbh_fast::sym_codes<BITS>(u, E), v0, v1);
+                    if constexpr (BITS == 3)
+                        upk2(sym_codes3x2(u, E), v0, v1);
+                    else
+                        upk2(rpbh_fast::sym_codes<BITS>(u, E), v0, v1);
                     cb[(2 * i) * S] = (uint8_t)__float_as_uint(v0);
                     cb[(2 * i + 1) * S] = (uint8_t)__float_as_uint(v1);
                 }
