@@ -118,8 +118,9 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def traffic_bytes(kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current source."""
+def traffic_bytes(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` in `workload` from the committed ncu summary, if one was
+    taken on that workload and on the current source."""
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
@@ -133,8 +134,9 @@ def traffic_bytes(kernel: str):
     with open(p) as f:
         for line in f:
             parts = line.split()
-            if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == sha:
-                return float(parts[3])
+            if (len(parts) >= 5 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload
+                    and parts[2] == sha):
+                return float(parts[4])
     return None
 
 
@@ -798,12 +800,12 @@ def run_ours(args):
         tpeak, tkind = measured_tensor_peak()
         tflops = wl.flops_per_launch[dom] / (per_kernel[dom]["avg_us"] * 1e-6) / 1e12
         roofline = {"bound": "tensor", "kernel": dom, "achieved": tflops, "peak": tpeak, "peak_kind": tkind,
-                    "unit": "TFLOP/s", "frac": tflops / tpeak, "traffic": traffic_bytes(dom),
+                    "unit": "TFLOP/s", "frac": tflops / tpeak, "traffic": traffic_bytes(dom, args.workload),
                     "algorithmic_flops_per_launch": wl.flops_per_launch[dom],
                     "algorithmic_bytes_per_launch": wl.bytes_per_launch[dom]}
     else:
         roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                    "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_bytes(dom),
+                    "unit": "GB/s", "frac": achieved / peak, "traffic": traffic_bytes(dom, args.workload),
                     "algorithmic_bytes_per_launch": wl.bytes_per_launch[dom]}
     if rank == 0:
         line = {

@@ -28,11 +28,13 @@ def test_traffic_is_reported_only_for_the_source_it_was_taken_on():
            "rpbh_rotate": "rpbh_lanes.cu", "rpbh_linear": "rpbh_linear.cu", "tq3_attention": "tq3_attn.cu"}
     lines = [l.split() for l in open(os.path.join(ROOT, "profiles", "traffic.txt")) if l.strip() and not l.startswith("#")]
     assert lines
-    for name, sha, _, value in lines:
+    for name, workload, sha, _, value in lines:
+        assert workload in bench.WORKLOADS
         cur = hashlib.sha256(open(os.path.join(ROOT, "weight_quantization_b200", "csrc", src[name]), "rb").read())
-        got = bench.traffic_bytes(name)
+        got = bench.traffic_bytes(name, workload)
         if cur.hexdigest()[:16] == sha:
             assert got == float(value)
         else:
             assert got is None
-    assert bench.traffic_bytes("no_such_kernel") is None
+    assert bench.traffic_bytes("no_such_kernel", "kv") is None
+    assert bench.traffic_bytes("tq3_decode", "no_such_workload") is None
