@@ -70,6 +70,8 @@ def test_quantize_llm_weight_full_size(wq, oracle, bits):
     w = _llm_weight()
     st, _, _ = _quantize_and_check(wq, oracle, w, True, 11008, bits)
     print("rpbh quantize C4", bits, st)
+    # the same fp32 steps as the oracle, with fp64 norms: every code and every bf16 norm matches
+    assert st["code_mismatches"] == 0 and st["bytes_equal"] and st["norms_equal"] == w.shape[0], st
 
 
 _W4 = None
@@ -88,6 +90,7 @@ def test_quantize_dit_weights_full_size(wq, oracle, rows):
     w = inputs.dit_weight(rows)
     st, _, _ = _quantize_and_check(wq, oracle, w, True, 3072, 3)
     print("rpbh quantize C5", rows, st)
+    assert st["code_mismatches"] == 0 and st["bytes_equal"] and st["norms_equal"] == rows, st
 
 
 @pytest.mark.parametrize("d,rows,bits", [(96, 7, 2), (192, 3, 3), (1024, 5, 3), (3072, 33, 4), (11008, 4, 3),
