@@ -62,6 +62,7 @@ def test_quantize_small(wq, oracle, d, rows, bits, is_bf16):
     if is_bf16:
         w = inputs.to_bf16_bits(torch.from_numpy(w))
     st, _, _ = _quantize_and_check(wq, oracle, w, is_bf16, d, bits)
+    assert st["code_mismatches"] == 0 and st["bytes_equal"] and st["norms_equal"] == rows, st
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4])
