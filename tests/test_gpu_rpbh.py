@@ -236,11 +236,13 @@ def test_requantize_norm_dtype(wq, oracle, d, rows, bits, w_bf16, norm_bf16):
     assert norms.dtype == ndt and norms.shape == (rows,)
     st, ref_packed, ref_norms = parity.check_rpbh_quantize(oracle, w, w_bf16, perm, signs, d & -d, cb, bits,
                                                             packed.cpu().numpy())
+    assert st["code_mismatches"] == 0 and st["bytes_equal"], st
     if norm_bf16:
+        # one nearest-even rounding of the fp32 norm, which equals the oracle's
         ref16 = oracle.f32_array_to_bf16(ref_norms).astype(np.int64)
-        assert np.all(np.abs(_np16(norms).astype(np.int64) - ref16) <= 1)
+        assert np.array_equal(_np16(norms).astype(np.int64), ref16)
     else:
-        parity.check_norms(norms.cpu().numpy(), ref_norms)
+        assert np.array_equal(norms.cpu().numpy(), ref_norms)
     # the same codes as rpbh_quantize_weight, whose norms follow the weight's dtype
     p2, n2 = wq.rpbh_quantize_weight(_t(w, w_bf16), perm_d, signs_d, bits, cb)
     assert torch.equal(p2, packed)
