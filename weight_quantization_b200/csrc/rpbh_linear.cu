@@ -85,6 +85,71 @@ __device__ __forceinline__ uint32_t code_at(const uint32_t (&W)[2 * BITS], int i
     return __funnelshift_l(W[q + 1], W[q], r + BITS - 32);
 }
 
+// The lookup of 2- and 3-bit codes by byte permutes, on the integer pipe: the 2^BITS bf16 entries
+// split into an 8-byte table of their low bytes and one of their high bytes; a byte permute whose
+// selector nibble k holds a code copies that code's byte into byte k of the result, so two permutes
+// look up four codes and two more interleave the low and high bytes into bf16 pairs.
+struct ByteTables {
+    uint32_t lo0, lo1, hi0, hi1;  // byte k of lo0 (k < 4) / lo1 (k >= 4): low byte of entry k
+};
+
+__device__ __forceinline__ ByteTables byte_tables(const CodebookBf16 &cb, int entries) {
+    ByteTables t = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const uint32_t e = k < entries ? cb.c[k] : 0u;
+        if (k < 4) {
+            t.lo0 |= (e & 0xffu) << (8 * k);
+            t.hi0 |= (e >> 8) << (8 * k);
+        } else {
+            t.lo1 |= (e & 0xffu) << (8 * (k - 4));
+            t.hi1 |= (e >> 8) << (8 * (k - 4));
+        }
+    }
+    return t;
+}
+
+// The four BITS-bit codes of x (4 BITS bits, first code in the top bits, nothing above) as the
+// four nibbles of a byte-permute selector, the last code in nibble 0. Two steps, each an exact
+// multiply-add that moves the upper half of every field group up: for 3 bits
+// (x & 0x3f) | (x & 0xfc0) << 2, then (y & 0x0707) | (y & 0x3838) << 1.
+template <int BITS>
+__device__ __forceinline__ uint32_t spread4(uint32_t x) {
+    if constexpr (BITS == 3) {
+        const uint32_t y = (x & 0xfc0u) * 3u + x;
+        return (y & 0x3838u) + y;
+    } else {
+        const uint32_t y = (x & 0xf0u) * 15u + x;
+        return (y & 0x0c0cu) * 3u + y;
+    }
+}
+
+// Codes 8j .. 8j + 7 of a chunk (stream bytes BITS j .. BITS j + BITS - 1 of the little-endian
+// words R) as four bf16 pairs, code 8j in the low half of w[0].
+template <int BITS>
+__device__ __forceinline__ void lookup8(const uint32_t (&R)[2 * BITS], int j, const ByteTables &t, uint32_t (&w)[4]) {
+    uint32_t xa, xb;  // codes 8j .. 8j + 3 and 8j + 4 .. 8j + 7
+    if constexpr (BITS == 3) {
+        const int b0 = 3 * j, q = b0 >> 2, u = b0 & 3;
+        // the group's three bytes, first in bits 16 .. 23 (byte 3 of the result is not used)
+        const uint32_t g = __byte_perm(R[q], q + 1 < 2 * BITS ? R[q + 1] : 0u, (u + 2) | ((u + 1) << 4) | (u << 8));
+        xa = (g >> 12) & 0xfffu;
+        xb = g & 0xfffu;
+    } else {
+        const int b0 = 2 * j, q = b0 >> 2, u = b0 & 3;
+        const uint32_t g = __byte_perm(R[q], 0u, (u + 1) | (u << 4));
+        xa = (g >> 8) & 0xffu;
+        xb = g & 0xffu;
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t sel = spread4<BITS>(h ? xb : xa);
+        const uint32_t L = __byte_perm(t.lo0, t.lo1, sel), H = __byte_perm(t.hi0, t.hi1, sel);
+        w[2 * h] = __byte_perm(L, H, 0x6273);      // first and second code of the four
+        w[2 * h + 1] = __byte_perm(L, H, 0x4051);  // third and fourth
+    }
+}
+
 template <int BITS, bool kNormBf16, int TN>
 __global__ void __launch_bounds__(kThreads, 1)
     linear_kernel(const uint8_t *__restrict__ packed, const void *__restrict__ row_norms, int out_f, int d,
@@ -169,8 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = n0 + p;
         const bool valid = n < out_f;
         const uint8_t *const src = packed + (int64_t)(valid ? n : 0) * (d / 8 * BITS);
-        // lane l holds the bf16 centroid l mod 2^bits: a shuffle from the lane named by a code is the lookup
+        // 4 bits: lane l holds the bf16 centroid l mod 16, and a shuffle from the lane named by a code
+        // is the lookup; 2 and 3 bits: byte permutes
         const uint32_t cbv = cb.c[lane & ((1 << BITS) - 1)];
+        const ByteTables tabs = byte_tables(cb, 1 << BITS);
         unsigned char *const rowA = base + kOffA + (p >> 7) * kAHalf + (p & 127) * 128;
         const int sw = p & 7;
         // the code bytes of chunk c + 2 are loaded while chunk c is unpacked (two register sets
@@ -190,11 +257,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) ok = mbar_wait_bounded(&empty[s], (uint32_t)(c / kStages - 1) & 1u, kMaxPolls);
                 if (!__all_sync(0xffffffffu, ok)) fault = true;
             }
-            // the chunk's 8 * BITS code bytes, as big-endian words
-            uint32_t W[2 * BITS];
+            // the chunk's 8 * BITS code bytes, as little-endian words (R) and as big-endian words (W)
+            uint32_t R[2 * BITS], W[2 * BITS];
 #pragma unroll
             for (int q = 0; q < BITS; ++q) {
                 const uint2 v = (c & 1) ? raw[1][q] : raw[0][q];
+                R[2 * q] = v.x;
+                R[2 * q + 1] = v.y;
                 W[2 * q] = __byte_perm(v.x, 0u, 0x0123);
                 W[2 * q + 1] = __byte_perm(v.y, 0u, 0x0123);
             }
@@ -204,13 +273,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fetch(c + 2, raw[0]);
             unsigned char *const A = rowA + s * kABytes;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {  // 16-byte chunk j: k = 8j .. 8j + 7
+            for (int j = 0; j < 8; ++j) {  // 16-byte chunk j: k = 8j .. 8j + 7 (rows past out_features: never stored)
                 uint32_t w4[4];
+                if constexpr (BITS == 4) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint32_t lo = __shfl_sync(0xffffffffu, cbv, (int)code_at<BITS>(W, 8 * j + 2 * u));
-                    const uint32_t hi = __shfl_sync(0xffffffffu, cbv, (int)code_at<BITS>(W, 8 * j + 2 * u + 1));
-                    w4[u] = __byte_perm(lo, hi, 0x5410);  // (rows past out_features: never stored)
+                    for (int u = 0; u < 4; ++u) {
+                        const uint32_t lo = __shfl_sync(0xffffffffu, cbv, (int)code_at<BITS>(W, 8 * j + 2 * u));
+                        const uint32_t hi = __shfl_sync(0xffffffffu, cbv, (int)code_at<BITS>(W, 8 * j + 2 * u + 1));
+                        w4[u] = __byte_perm(lo, hi, 0x5410);
+                    }
+                } else {
+                    lookup8<BITS>(R, j, tabs, w4);
                 }
                 *reinterpret_cast<uint4 *>(A + ((j ^ sw) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
             }
