@@ -228,10 +228,12 @@ class KVWorkload:
         self.table = torch.randperm(n // self.page, generator=g).to(torch.int32).to(dev)
         pos = torch.arange(n, dtype=torch.int64)
         self.slots = (self.table.cpu().to(torch.int64)[pos // self.page] * self.page + pos % self.page).to(dev)
+        # the same cache as fp32 (268 MB, larger than L2), for the fp32-input encoder beside the step
+        self.x32 = self.x[0].float()
         self.kernels = ["tq3_encode", "tq3_decode"]
         self.bytes_per_launch = {"tq3_encode": 312 * n, "tq3_decode": 312 * n, "tq3_encode_aos": 312 * n,
                                  "tq3_decode_aos": 312 * n, "tq3_encode_slots": 320 * n,
-                                 "tq3_decode_paged": (312 + 4 / self.page) * n}
+                                 "tq3_decode_paged": (312 + 4 / self.page) * n, "tq3_encode_fp32": 568 * n}
         self.l2 = (f"cache (134 MB) larger than L2; records rotate over {R} sets: launch k encodes into "
                    f"set k % {R} and decodes set (k + 1) % {R}, written {R - 1} launches earlier")
 
@@ -253,10 +255,13 @@ class KVWorkload:
         return [("tq3_encode", 1, self._encode), ("tq3_decode", 1, self._decode)]
 
     def extras(self):
-        """Kernels timed beside the step (not part of it): the bit-exact encoder on the same cache and
-        the codec on 56-byte records."""
+        """Kernels timed beside the step (not part of it): the bit-exact encoder on the same cache, the
+        encoder on the cache as fp32 input, and the codec on 56-byte records."""
         o, R = self.ops, self.RSETS
         return [("tq3_encode_exact", 1, lambda k: self._encode(k, exact=True)),
+                ("tq3_encode_fp32", 1, lambda k: o.tq3_encode(self.x32, self.mask, self.packed[k % R].view(-1, 1, 48),
+                                                               self.norms[k % R].view(-1, 1),
+                                                               self.scales[k % R].view(-1, 1))),
                 ("tq3_encode_aos", 1, lambda k: o.tq3_encode_aos(self.x[0], self.mask, records=self.recs[k % R])),
                 ("tq3_decode_aos", 1, lambda k: o.tq3_decode_aos(self.recs[(k + 1) % R], self.mask,
                                                                  out_dtype=torch.bfloat16, out=self.out[0])),

@@ -1,8 +1,9 @@
 """Host checks of the constants the fast TQ3 encoders decide with (page "tq3_core.py",
 _quantize_to_indices: searchsorted against TQ3_BOUNDARIES, right=False).
 
-The tensor-core encoder computes the index of a scaled coefficient x in [-1, 1] as 3 + ceil(Q(x)),
-Q(x) = q1 x + q3 x^3 + q5 x^5, with the three fp32 coefficients written in its source. These tests
+Both fast encoders (the tensor-core one for bf16 input, the one-thread-per-vector one for fp32)
+compute the index of a scaled coefficient x in [-1, 1] as 3 + ceil(Q(x)),
+Q(x) = q1 x + q3 x^3 + q5 x^5, with the three fp32 coefficients written in the shared TQ3 header. These tests
 read the coefficients from the source and check, in fp32 arithmetic emulated with numpy, what that
 rule relies on: Q passes through 1, 2, 3 at the positive boundaries, is odd and increasing, stays
 below 4 at x = 1, and its evaluation (Horner in x^2, the last step an exact product followed by
@@ -15,7 +16,7 @@ import numpy as np
 
 from conftest import ROOT
 
-SRC = os.path.join(ROOT, "weight_quantization_b200", "csrc", "tq3_mma.cu")
+SRC = os.path.join(ROOT, "weight_quantization_b200", "csrc", "tq3_common.cuh")
 B = np.array([-0.7992, -0.4824, -0.2304, 0.0, 0.2304, 0.4824, 0.7992], dtype=np.float32).astype(np.float64)
 
 

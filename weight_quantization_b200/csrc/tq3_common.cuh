@@ -50,6 +50,28 @@ inline bool is_default(const SignMask &m) {
     return true;
 }
 
+// fma.rp.f32x2: two fused multiply-adds rounded towards +infinity.
+__device__ __forceinline__ f32x2 fma2_rp(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 r;
+    asm("fma.rp.f32x2 %0,%1,%2,%3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// The decision polynomial. With x = xs the scaled coefficient in [-1, 1], the page's index is
+// #{j : B_j < x} over TQ3_BOUNDARIES B = (-b2, -b1, -b0, 0, b0, b1, b2). Let Q be the odd quintic
+// Q(x) = q1 x + q3 x^3 + q5 x^5 with Q(b_k) = k + 1 for the three positive boundaries (solved in
+// fp64 from the fp32 boundary values, then rounded to fp32). Q is increasing on [-1, 1] (Q' >= 1.97)
+// and Q(1) = 3.46 < 4, so #{j : B_j < x} = 3 + ceil(Q(x)) for every x in [-1, 1]: at a boundary
+// ceil(Q) is exactly the integer k + 1, which puts the value in the lower bucket as searchsorted
+// does, and an exact 0 gives index 3. The ceiling costs nothing: the last Horner step
+// h x + (2^23 + 4) is one fma rounded towards +infinity, whose result (between 2^23 and 2^24) is the
+// integer 2^23 + 4 + ceil(h x). The fp32 evaluation moves each boundary by at most about 1.3e-7 in
+// x, which the parity rule's 1e-6 tie window absorbs. Both fast encoders decide their
+// indices this way.
+__device__ __forceinline__ float q_coef(int k) {
+    return __uint_as_float(k == 1 ? 0x408cce16u : k == 3 ? 0xbf91bb0au : 0x3e4acae9u);
+}
+
 // fp32(1.0 / math.sqrt(128)), the post-multiplier of _fwht_inplace.
 __device__ __forceinline__ float fwht_post() { return __uint_as_float(0x3DB504F3u); }
 

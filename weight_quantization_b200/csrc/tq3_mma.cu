@@ -108,27 +108,6 @@ __device__ __forceinline__ void build_b(unsigned char *B, const SignMask &mask, 
     }
 }
 
-// fma.rp.f32x2: two fused multiply-adds rounded towards +infinity.
-__device__ __forceinline__ f32x2 fma2_rp(f32x2 a, f32x2 b, f32x2 c) {
-    f32x2 r;
-    asm("fma.rp.f32x2 %0,%1,%2,%3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
-// The decision polynomial. With x = xs the scaled coefficient in [-1, 1], the page's index is
-// #{j : B_j < x} over TQ3_BOUNDARIES B = (-b2, -b1, -b0, 0, b0, b1, b2). Let Q be the odd quintic
-// Q(x) = q1 x + q3 x^3 + q5 x^5 with Q(b_k) = k + 1 for the three positive boundaries (solved in
-// fp64 from the fp32 boundary values, then rounded to fp32). Q is increasing on [-1, 1] (Q' >= 1.97)
-// and Q(1) = 3.46 < 4, so #{j : B_j < x} = 3 + ceil(Q(x)) for every x in [-1, 1]: at a boundary
-// ceil(Q) is exactly the integer k + 1, which puts the value in the lower bucket as searchsorted
-// does, and an exact 0 gives index 3. The ceiling costs nothing: the last Horner step
-// h x + (2^23 + 4) is one fma rounded towards +infinity, whose result (between 2^23 and 2^24) is the
-// integer 2^23 + 4 + ceil(h x). The fp32 evaluation moves each boundary by at most about 1.3e-7 in
-// x, which the parity rule's 1e-6 tie window absorbs.
-__device__ __forceinline__ float q_coef(int k) {
-    return __uint_as_float(k == 1 ? 0x408cce16u : k == 3 ? 0xbf91bb0au : 0x3e4acae9u);
-}
-
 // Indices of one 32-column piece (elements 32c .. 32c + 31, groups 4c .. 4c + 3) packed as the
 // record's bytes 12c .. 12c + 11, three little-endian words (_pack_3bit: group i is bytes
 // 3i .. 3i + 2). nr = -1 / T turns the accumulator's z = -fwht into x = z * nr. Group q is
@@ -136,7 +115,8 @@ __device__ __forceinline__ float q_coef(int k) {
 // below 2^24, so the words are exact.
 __device__ __forceinline__ void bucket_piece(const float (&z)[32], float nr, uint32_t &o0, uint32_t &o1, uint32_t &o2) {
     const f32x2 NR = pk2(nr, nr);
-    const f32x2 Q1 = pk2(q_coef(1), q_coef(1)), Q3 = pk2(q_coef(3), q_coef(3)), Q5 = pk2(q_coef(5), q_coef(5));
+    const f32x2 Q1 = pk2(tq3::q_coef(1), tq3::q_coef(1)), Q3 = pk2(tq3::q_coef(3), tq3::q_coef(3)),
+               Q5 = pk2(tq3::q_coef(5), tq3::q_coef(5));
     const f32x2 KK = pk2(8388612.0f, 8388612.0f), NC = pk2(-8388609.0f, -8388609.0f);
     f32x2 W[4];
 #pragma unroll
@@ -150,7 +130,7 @@ __device__ __forceinline__ void bucket_piece(const float (&z)[32], float nr, uin
             const f32x2 x = mul2(pk2(z[2 * i], z[2 * i + 1]), NR);
             const f32x2 x2 = mul2(x, x);
             const f32x2 h = fma2(fma2(Q5, x2, Q3), x2, Q1);
-            const f32x2 idx = add2(fma2_rp(h, x, KK), NC);  // 3 + ceil(Q(x))
+            const f32x2 idx = add2(tq3::fma2_rp(h, x, KK), NC);  // 3 + ceil(Q(x))
             W[gg] = fma2(w8, idx, W[gg]);
         }
     uint32_t g4[4];

@@ -16,11 +16,11 @@
 // Encoder numerics. The page normalises x, transforms, scales by the absmax and compares
 // xs = RN(RN(y c) / scale) with the boundaries. In exact arithmetic xs_i = z_i / max|z| with
 // z = fwht(D x) (the norm and c cancel), unless the 1e-8 floor on the scale is active. This kernel
-// therefore transforms the unnormalised input and decides |xs_i| > b as |z_i| > b * T with
-// T = max|z| (T = 1e-8 * norm * sqrt(128) when the floor is active). Each decision is exact for the
-// fp32 values it compares; the only difference from the page's own rounding sequence is a few
-// units in the last place of xs, so an index can differ from the step-by-step result only for a
-// coefficient within about 1e-6 of a boundary (ties included). Norms come from an fp32 sum of
+// therefore transforms the unnormalised input, forms x_i = RN(z_i RN(1 / T)) with T = max|z|
+// (T = 1e-8 * norm * sqrt(128) when the floor is active) and takes the index from the decision
+// polynomial, 3 + ceil(Q(x_i)) (tq3_common.cuh). The rounding of x and the polynomial's fp32
+// evaluation move each boundary by a few 1e-7 in xs, so an index can differ from the step-by-step
+// result only for a coefficient within 1e-6 of a boundary (ties included). Norms come from an fp32 sum of
 // squares (within 1e-6 relative), scales = max(RN(RN(max|z| / norm) * c), 1e-8). A vector whose
 // fp32 sum of squares is not finite (|x| beyond about 1e19, where the unnormalised transform can
 // itself overflow although the page's normalised one does not) is encoded by the page's steps
@@ -107,9 +107,6 @@ struct EncGeo {
     static constexpr int kFlipOff = kBarOff + 64;
     static constexpr int kSmem = 1024 + kFlipOff + 4 * kFlipWords;
 };
-
-// The positive TQ3_BOUNDARIES (fp32); the others are their negatives and 0.
-__device__ __forceinline__ float edge(int k) { return k == 0 ? 0.2304f : k == 1 ? 0.4824f : 0.7992f; }
 
 // kLay (tq3::Layout): kSoA writes packed, norms and scales; kAoS writes 56-byte records at
 // `packed`; kPool writes record v to slot pm.index[v] of the pool at `packed` (here and in
@@ -256,40 +253,26 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         const float sraw = __fmul_rn(__fdiv_rn(m, nrm), post);
         const float scale = fmaxf(sraw, 1e-8f);
         const float T = (sraw >= 1e-8f) ? m : __fmul_rn(__fmul_rn(1e-8f, nrm), 11.3137085f);
-        const float t0 = __fmul_rn(edge(0), T), t1 = __fmul_rn(edge(1), T), t2 = __fmul_rn(edge(2), T);
-        // M = 1 / ulp(t0): (|z| - t) M is >= 1 whenever |z| > t >= t0, and exact near t (Sterbenz)
-        const uint32_t Mb = (277u - ((__float_as_uint(t0) >> 23) & 0xffu)) << 23;
-        const float M = __uint_as_float(Mb);
-        const float K0 = -__fmul_rn(t0, M), K1 = -__fmul_rn(t1, M), K2 = -__fmul_rn(t2, M);
-
-        // idx = 3.5 + sgn(u) (c + 0.5), c = #{k : |z| > t_k}, u = -z (sgn(+-0) = -1), as 8^j-weighted
-        // fp32 words of 8 indices; every partial sum is an integer (or the initial half-integer)
-        // below 2^24, so the words are exact
+        // the indices by the decision polynomial (tq3::q_coef): x = u / T with u = -z, the true
+        // coefficient, then idx = 3 + ceil(Q(x)), accumulated as 8^j-weighted fp32 words (exact
+        // integers below 2^24); the low half of W[g] is group g, the high half group g + 8
+        const f32x2 NR = pk2(-__frcp_rn(T), -__frcp_rn(T));
+        const f32x2 Q1 = pk2(tq3::q_coef(1), tq3::q_coef(1)), Q3 = pk2(tq3::q_coef(3), tq3::q_coef(3)),
+                    Q5 = pk2(tq3::q_coef(5), tq3::q_coef(5));
+        const f32x2 KK = pk2(8388612.0f, 8388612.0f), NC = pk2(-8388609.0f, -8388609.0f);
         f32x2 W[8];
 #pragma unroll
-        for (int g = 0; g < 8; ++g) W[g] = pk2(8388607.5f, 8388607.5f);  // sum_j 3.5 * 8^j
-        const f32x2 HALF = pk2(0.5f, 0.5f);
+        for (int g = 0; g < 8; ++g) W[g] = 0ull;
 #pragma unroll
         for (int kk = 0; kk < 64; ++kk) {
-            // slot-major order: consecutive steps update different words (independent chains);
-            // every word still starts with its slot-0 half-term
+            // slot-major order: consecutive steps update different words (independent chains)
             const int j = kk >> 3, k = 8 * (kk & 7) + j;
-            const uint32_t w8n = 0x80000000u | ((127u + 3u * j) << 23);  // bits of -8^j
-            float za, zb;
-            upk2(P[k], za, zb);
-            const uint32_t ha = __float_as_uint(za) & 0x80000000u, hb = __float_as_uint(zb) & 0x80000000u;
-            const float sMa = __uint_as_float(ha | Mb), sMb = __uint_as_float(hb | Mb);
-            const f32x2 w2 = pk2(__uint_as_float(ha ^ w8n), __uint_as_float(hb ^ w8n));
-            W[k >> 3] = fma2(w2, HALF, W[k >> 3]);
-            W[k >> 3] = fma2(w2,
-                             pk2(__saturatef(__fmaf_rn(za, sMa, K0)), __saturatef(__fmaf_rn(zb, sMb, K0))),
-                             W[k >> 3]);
-            W[k >> 3] = fma2(w2,
-                             pk2(__saturatef(__fmaf_rn(za, sMa, K1)), __saturatef(__fmaf_rn(zb, sMb, K1))),
-                             W[k >> 3]);
-            W[k >> 3] = fma2(w2,
-                             pk2(__saturatef(__fmaf_rn(za, sMa, K2)), __saturatef(__fmaf_rn(zb, sMb, K2))),
-                             W[k >> 3]);
+            const float w8s = __uint_as_float((127u + 3u * j) << 23);  // 8^j
+            const f32x2 x = mul2(P[k], NR);
+            const f32x2 x2 = mul2(x, x);
+            const f32x2 h = fma2(fma2(Q5, x2, Q3), x2, Q1);
+            const f32x2 idx = add2(tq3::fma2_rp(h, x, KK), NC);  // 3 + ceil(Q(x))
+            W[k >> 3] = fma2(pk2(w8s, w8s), idx, W[k >> 3]);
         }
         const int64_t v = (blockIdx.x + it * gridDim.x) * kTile + tid;
         if (v < n_vec) {
