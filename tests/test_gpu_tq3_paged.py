@@ -86,7 +86,8 @@ def _records_of(table, page_size, n_vec):
     return table[pos // page_size].astype(np.int64) * page_size + pos % page_size
 
 
-@pytest.mark.parametrize("page_size,n_pages_pool,n_vec", [(1, 500, 333), (16, 97, 16 * 60 + 7), (32, 64, 32 * 40),
+@pytest.mark.parametrize("page_size,n_pages_pool,n_vec", [(1, 500, 333), (4, 300, 4 * 250 + 3), (8, 200, 8 * 150 + 6),
+                                                          (16, 97, 16 * 60 + 7), (32, 64, 32 * 40),
                                                           (256, 40, 256 * 23 + 129), (4096, 12, 4096 * 9 + 5)])
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
 def test_decode_paged_bit_exact(wq, oracle, page_size, n_pages_pool, n_vec, out_dtype):

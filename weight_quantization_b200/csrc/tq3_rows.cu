@@ -403,8 +403,22 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
     int64_t tile = blockIdx.x;
     const bool pf_ok = ((reinterpret_cast<uintptr_t>(packed) | reinterpret_cast<uintptr_t>(norms) |
                          reinterpret_cast<uintptr_t>(scales)) & 15) == 0;
+    // Paged pool: the records of a tile two rounds ahead are prefetched page by page. With pages of
+    // 4 to 16 records a tile covers 32 >> shift whole pages (tiles start on multiples of 32), lane l
+    // taking page l; with 32 or more, one page, lane 0. A lane reads its page-table entry one round
+    // before the prefetch that needs it, so no lane waits on that read.
+    const int pf_lanes = kLay != tq3::kPool ? 0 : pm.shift >= 5 ? 1 : pm.shift >= 2 ? (kTile >> pm.shift) : 0;
+    auto page_entry = [&](int64_t t) -> int32_t {  // this lane's page-table entry for tile t, or -1
+        if constexpr (kLay == tq3::kPool) {
+            const int64_t first = pm.shift >= 5 ? 0 : (int64_t)tid << pm.shift;
+            if (tid < pf_lanes && t < n_tiles && t * kTile + first < n_vec)
+                return __ldg(static_cast<const int32_t *>(pm.index) + ((pm.v0 + t * kTile + first) >> pm.shift));
+        }
+        return -1;
+    };
     pdl_wait();  // the records may come from the kernel before this one
     Rec cur = load_rec<kLay>(packed, norms, scales, n_vec, tile * kTile + tid, pm);
+    int32_t pe = page_entry(tile + 2 * (int64_t)gridDim.x);
     for (int it = 0; tile < n_tiles; ++it, tile += gridDim.x) {
         // on its last tile the block lets the next kernel in the stream be scheduled: its set-up
         // overlaps this kernel's tail (it still waits for this kernel to finish before reading)
@@ -412,21 +426,27 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         const Rec nxt = load_rec<kLay>(packed, norms, scales, n_vec, (tile + gridDim.x) * kTile + tid, pm);
         // the records of the tile after that go into L2 now, so next iteration's load finds them
         // there (whole 16-byte units inside the arrays only)
-        if (tid == 0 && pf_ok && tile + 2 * gridDim.x < n_tiles) {
+        if constexpr (kLay == tq3::kPool) {
+            // a page's run of records starts on a 16-byte boundary and spans a multiple of 4 records:
+            // its first record is a multiple of 4 (page << shift, plus a multiple of 32 inside pages of
+            // 32 or more), and 56 * 4 = 224
+            const int32_t pe_next = page_entry(tile + 3 * (int64_t)gridDim.x);
+            if (pf_ok && pe >= 0) {
+                const int64_t v0 = (tile + 2 * gridDim.x) * kTile;
+                const int64_t cnt = (n_vec - v0 < kTile ? n_vec - v0 : kTile) & ~int64_t(3);
+                const int64_t first = pm.shift >= 5 ? 0 : (int64_t)tid << pm.shift;
+                const int64_t per = pm.shift >= 5 ? kTile : (int64_t(1) << pm.shift);
+                const int64_t c = cnt - first < per ? cnt - first : per;
+                const int64_t lp = pm.v0 + v0 + first;
+                const int64_t r0 = ((int64_t)pe << pm.shift) | (lp & ((int64_t(1) << pm.shift) - 1));
+                if (c > 0 && r0 + c <= pm.n_pool) bulk_prefetch_l2(packed + r0 * 56, (uint32_t)(c * 56));
+            }
+            pe = pe_next;
+        } else if (tid == 0 && pf_ok && tile + 2 * gridDim.x < n_tiles) {
             const int64_t v0 = (tile + 2 * gridDim.x) * kTile;
             const int64_t cnt = (n_vec - v0 < kTile ? n_vec - v0 : kTile) & ~int64_t(3);
             if (cnt > 0) {
-                if constexpr (kLay == tq3::kPool) {
-                    // with pages of 32 records or more a tile lies inside one page, so its records
-                    // are contiguous in the pool (and start on a 16-byte boundary)
-                    if (pm.shift >= 5) {
-                        const int64_t lp = pm.v0 + v0;
-                        const int32_t page = __ldg(static_cast<const int32_t *>(pm.index) + (lp >> pm.shift));
-                        const int64_t r0 = ((int64_t)page << pm.shift) | (lp & ((int64_t(1) << pm.shift) - 1));
-                        if (page >= 0 && r0 + cnt <= pm.n_pool)
-                            bulk_prefetch_l2(packed + r0 * 56, (uint32_t)(cnt * 56));
-                    }
-                } else if constexpr (kLay == tq3::kAoS) {
+                if constexpr (kLay == tq3::kAoS) {
                     bulk_prefetch_l2(packed + v0 * 56, (uint32_t)(cnt * 56));
                 } else {
                     bulk_prefetch_l2(packed + v0 * 48, (uint32_t)(cnt * 48));
