@@ -331,11 +331,15 @@ struct Rec {
     float n, s;
 };
 
-// Record of logical vector p (launch-relative) through the page table, or -1 (and the fault bit)
-// for an entry outside the pool.
-__device__ __forceinline__ int64_t pool_record(const tq3::PoolMap &pm, int64_t p) {
+// Page-table entry of logical vector p (launch-relative, inside the launch).
+__device__ __forceinline__ int32_t page_of(const tq3::PoolMap &pm, int64_t p) {
+    return __ldg(static_cast<const int32_t *>(pm.index) + ((pm.v0 + p) >> pm.shift));
+}
+
+// Record of logical vector p (launch-relative) whose page-table entry is `page`, or -1 (and the
+// fault bit) for an entry outside the pool.
+__device__ __forceinline__ int64_t pool_record(const tq3::PoolMap &pm, int64_t p, int32_t page) {
     const int64_t lp = pm.v0 + p;
-    const int32_t page = __ldg(static_cast<const int32_t *>(pm.index) + (lp >> pm.shift));
     const int64_t r = ((int64_t)page << pm.shift) | (lp & ((int64_t(1) << pm.shift) - 1));
     if (page < 0 || r >= pm.n_pool) {
         atomicOr(&g_fault, tq3::kFaultPoolIndex);
@@ -344,14 +348,16 @@ __device__ __forceinline__ int64_t pool_record(const tq3::PoolMap &pm, int64_t p
     return r;
 }
 
+// The record of vector v (launch-relative; zeros past n_vec). In the pool layout `page` is v's
+// page-table entry, read ahead by the caller.
 template <int kLay>
 __device__ __forceinline__ Rec load_rec(const uint8_t *__restrict__ packed, const float *__restrict__ norms,
                                         const float *__restrict__ scales, int64_t n_vec, int64_t v,
-                                        const tq3::PoolMap &pm) {
+                                        const tq3::PoolMap &pm, int32_t page) {
     Rec r;
     int64_t at = v < n_vec ? v : -1;
     if constexpr (kLay == tq3::kPool)
-        if (at >= 0) at = pool_record(pm, v);
+        if (at >= 0) at = pool_record(pm, v, page);
     if (at >= 0) {
         if constexpr (kLay != tq3::kSoA) {  // a 56-byte record is 8-byte aligned
             const uint8_t *p = packed + at * 56;
@@ -416,14 +422,25 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
         }
         return -1;
     };
+    // pool layout: the page-table entry of this thread's vector in a tile, read one round before
+    // the record load that needs it
+    auto vec_page = [&](int64_t t) -> int32_t {
+        if constexpr (kLay == tq3::kPool) {
+            const int64_t v = t * kTile + tid;
+            if (v < n_vec) return page_of(pm, v);
+        }
+        return -1;
+    };
     pdl_wait();  // the records may come from the kernel before this one
-    Rec cur = load_rec<kLay>(packed, norms, scales, n_vec, tile * kTile + tid, pm);
+    Rec cur = load_rec<kLay>(packed, norms, scales, n_vec, tile * kTile + tid, pm, vec_page(tile));
+    int32_t pv = vec_page(tile + gridDim.x);
     int32_t pe = page_entry(tile + 2 * (int64_t)gridDim.x);
     for (int it = 0; tile < n_tiles; ++it, tile += gridDim.x) {
         // on its last tile the block lets the next kernel in the stream be scheduled: its set-up
         // overlaps this kernel's tail (it still waits for this kernel to finish before reading)
         if (tile + gridDim.x >= n_tiles) pdl_trigger();
-        const Rec nxt = load_rec<kLay>(packed, norms, scales, n_vec, (tile + gridDim.x) * kTile + tid, pm);
+        const Rec nxt = load_rec<kLay>(packed, norms, scales, n_vec, (tile + gridDim.x) * kTile + tid, pm, pv);
+        pv = vec_page(tile + 2 * (int64_t)gridDim.x);
         // the records of the tile after that go into L2 now, so next iteration's load finds them
         // there (whole 16-byte units inside the arrays only)
         if constexpr (kLay == tq3::kPool) {
