@@ -466,9 +466,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks)
                 if constexpr (kLay == tq3::kAoS) {
                     bulk_prefetch_l2(packed + v0 * 56, (uint32_t)(cnt * 56));
                 } else {
+                    // the packed bytes only: prefetching the tile's 128-byte runs of norms and
+                    // scales as well measured 2.2 us slower per launch on the KV cache
                     bulk_prefetch_l2(packed + v0 * 48, (uint32_t)(cnt * 48));
-                    bulk_prefetch_l2(norms + v0, (uint32_t)(cnt * 4));
-                    bulk_prefetch_l2(scales + v0, (uint32_t)(cnt * 4));
                 }
             }
         }
