@@ -54,6 +54,7 @@ constexpr int kMaxSplit = 8;   // CTAs per cluster (portable cluster size)
 constexpr int kMaxRows = 16;   // query rows per launch (chunk)
 constexpr int64_t kMaxRowsTotal = 1 << 20;  // query rows per head in one call
 constexpr int kThreads = 128;
+constexpr uint32_t kMaxPolls = 1u << 24;
 
 __device__ unsigned int g_fault;
 
@@ -99,6 +100,7 @@ struct Smem {
     float red[kWarps][kRows];      // per-warp partial maxima and sums
     float mrow[kRows], lrow[kRows];
     int valid[2][kKeys];           // per tile parity: 1 when the key exists and its records were found
+    uint64_t bar[2];               // bulk copies of a whole tile's key (0) and value (1) records
 };
 
 // Sign draw of element e: +1.0 or -1.0.
@@ -140,9 +142,41 @@ __global__ void __launch_bounds__(kThreads, 4)
 
     const int64_t n_tiles = (S + kKeys - 1) / kKeys;
     const int64_t t_begin = n_tiles * split / n_split, t_end = n_tiles * (split + 1) / n_split;
-    // the key (or value) records of keys tid + 128 k of a tile, by 8-byte asynchronous copies; the
-    // key pass also records which keys exist (parity b of the tile index)
+    // A whole tile of a contiguous cache is one run of kKeys records in global memory, laid out as
+    // the shared-memory buffer is: thread 0 copies it with one bulk copy per tensor (on the copy
+    // engine, not the load/store pipe), when the run starts on a 16-byte boundary (records are 56
+    // bytes, so head * S must be even). Other tiles take the per-thread copies below.
+    // (The 16-row form, already at its register limit, keeps the per-thread copies.)
+    constexpr bool kBulk = kRows <= 8;
+    const bool bulk_ok = kBulk && kv.table == nullptr &&
+                         ((reinterpret_cast<uintptr_t>(kv.k) | reinterpret_cast<uintptr_t>(kv.v)) & 15) == 0 &&
+                         ((head * S) & 1) == 0;
+    // Only a partial last tile is not bulk, so the bulk tiles are the CTA's tiles in order: tile t
+    // completes phase (t - t_begin) & 1 of each barrier.
+    auto is_bulk = [&](int64_t tile) { return bulk_ok && (tile + 1) * kKeys <= S; };
+    if constexpr (kBulk) {
+        if (tid == 0) {
+            mbar_init(&sm.bar[0], 1);
+            mbar_init(&sm.bar[1], 1);
+        }
+        __syncthreads();  // the barriers are initialised before the first copy is issued on them
+    }
+    // the key (or value) records of keys tid + 128 k of a tile, by 8-byte asynchronous copies (or
+    // one bulk copy); the key pass also records which keys exist (parity b of the tile index)
     auto fetch = [&](int64_t tile, bool values, int b) {
+        if (is_bulk(tile)) {
+            if (!values) {
+#pragma unroll
+                for (int k = 0; k < kKPT; ++k) sm.valid[b][tid + kThreads * k] = 1;
+            }
+            if (tid == 0) {
+                uint64_t *bar = &sm.bar[values ? 1 : 0];
+                mbar_expect_tx(bar, (uint32_t)(kKeys * 56));
+                bulk_load(values ? &sm.u.rec.v[0][0] : &sm.u.rec.k[0][0],
+                          (values ? kv.v : kv.k) + (head * S + tile * kKeys) * 56, (uint32_t)(kKeys * 56), bar);
+            }
+            return;
+        }
 #pragma unroll
         for (int k = 0; k < kKPT; ++k) {
             const int key = tid + kThreads * k;
@@ -196,7 +230,23 @@ __global__ void __launch_bounds__(kThreads, 4)
 
     for (int64_t tile = t_begin; tile < t_end; ++tile) {
         const int b = (int)((tile - t_begin) & 1);
-        cp_async_wait<0>();
+        if (is_bulk(tile)) {
+            const bool ok = mbar_wait_bounded(&sm.bar[0], (uint32_t)b, kMaxPolls) &&
+                            mbar_wait_bounded(&sm.bar[1], (uint32_t)b, kMaxPolls);
+            if (__syncthreads_or(!ok)) {
+                // a copy that did not complete in time: results void. Give it another bounded
+                // chance to land before the buffers are reused, then leave the tiles.
+                if (tid == 0) {
+                    atomicOr(&g_fault, 2u);
+                    mbar_wait_bounded(&sm.bar[0], (uint32_t)b, kMaxPolls);
+                    mbar_wait_bounded(&sm.bar[1], (uint32_t)b, kMaxPolls);
+                }
+                __syncthreads();
+                break;
+            }
+        } else {
+            cp_async_wait<0>();
+        }
         __syncthreads();  // this tile's records (and valid flags) are visible to every thread
         const uint32_t(*kr)[kWords] = sm.u.rec.k;
         const uint32_t(*vr)[kWords] = sm.u.rec.v;
@@ -265,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, 4)
                 if (lane == 0) sm.red[warp][r] = mx;
             }
         }
+        if (bulk_ok) fence_proxy_async_smem();  // these reads precede a bulk copy into the buffer
         __syncthreads();  // every thread is past its reads of the key records
         if (tile + 1 < t_end) fetch(tile + 1, false, b ^ 1);
 
@@ -346,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, 4)
                     for (int c = 0; c < 4; ++c) acc[c][rp] = fma2(cv[c], wj[rp], acc[c][rp]);
             }
         }
+        if (bulk_ok) fence_proxy_async_smem();  // these reads precede a bulk copy into the buffer
         __syncthreads();  // every thread is past its reads of the value records
         if (tile + 1 < t_end) fetch(tile + 1, true, b ^ 1);
     }
