@@ -305,7 +305,7 @@ wq_status wq_rpbh_codebook(int bits, int64_t d, float *out);
 /* wq_device_fault -- reads and clears the library's sticky device fault bits. A kernel whose
  * bounded wait runs out (which does not happen in normal operation) sets a bit and returns early,
  * leaving its outputs unspecified: bit 0 a TQ3 kernel waiting for a TMA tile, bit 1 an RPBH kernel
- * waiting for a row copy, bit 3 the tensor-core TQ3 encoder waiting for a tile or its product,
+ * waiting for a row copy or the CUDA-core attention waiting for a tile's records, bit 3 the tensor-core TQ3 encoder waiting for a tile or its product,
  * bit 4 rpbh_linear waiting for a tile, the unpacked weights or its product, bit 5 the self-test
  * wq_selftest_wait_timeout, bit 7 the tensor-core attention waiting for its product. Bit 6 is not a wait: tq3_encode_slots, tq3_decode_paged or
  * tq3_attention_paged met a slot or page-table entry outside the pool (that record was skipped,

@@ -25,7 +25,8 @@
 // that one shared-memory read of the rotated query serves kKPT keys; for the values, each lane owns
 // four rotated coordinates and each warp a quarter of the tile's keys, two query rows per packed
 // multiply-add, the warps' sums being added once at the end. The records of the next tile are
-// copied into shared memory asynchronously (8-byte cp.async) while the current one is processed.
+// copied into shared memory asynchronously while the current one is processed: a whole tile of a
+// contiguous cache by one bulk copy per tensor, other tiles by 8-byte cp.async.
 //
 // Records are addressed either contiguously ([heads][S] records) or through a page table over a
 // pool of records (the layout tq3_encode_slots writes): key j of head h is record
