@@ -49,6 +49,44 @@ def measured_peaks():
     return HBM_FALLBACK_GBS, "fallback"
 
 
+def host_cpu():
+    """The host's CPU model and the number of cores this process may run on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        nproc = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        nproc = os.cpu_count()
+    return {"cpu": model or "unknown", "nproc": nproc}
+
+
+class OneCore:
+    """Runs the single-threaded oracle pinned to one of this process's cores, when the host allows
+    it (`pinned` says whether it did); the affinity is restored afterwards."""
+
+    def __enter__(self):
+        self.saved, self.pinned = None, False
+        try:
+            self.saved = os.sched_getaffinity(0)
+            os.sched_setaffinity(0, {min(self.saved)})
+            self.pinned = True
+        except (AttributeError, OSError, ValueError):
+            pass
+        return self
+
+    def __exit__(self, *exc):
+        if self.pinned:
+            os.sched_setaffinity(0, self.saved)
+        return False
+
+
 def measured_tensor_peak():
     """Dense bf16 TFLOP/s measured on this machine (a cuBLAS burst), or the fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -828,8 +866,10 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, sample = wl.oracle_rate(args.cpu_seconds)
-        cpu = {"value": rate, "unit": wl.unit, "cores": 1, "kind": "oracle", "sample": sample}
+        with OneCore() as pin:
+            rate, sample = wl.oracle_rate(args.cpu_seconds)
+        cpu = {"value": rate, "unit": wl.unit, "cores": 1, "kind": "oracle", "sample": sample,
+               "pinned": pin.pinned, **host_cpu()}
 
     if getattr(wl, "bound", "hbm") == "tensor":
         tpeak, tkind = measured_tensor_peak()
@@ -889,13 +929,14 @@ def run_reference(args):
             return chunk
     else:
         raise SystemExit(f"--impl reference supports the default workload only, not {args.workload}")
-    for i in range(args.warmup):
-        step(i)
-    t0 = time.perf_counter()
-    units = 0
-    for i in range(args.steps):
-        units += step(args.warmup + i)
-    dt = time.perf_counter() - t0
+    with OneCore() as pin:
+        for i in range(args.warmup):
+            step(i)
+        t0 = time.perf_counter()
+        units = 0
+        for i in range(args.steps):
+            units += step(args.warmup + i)
+        dt = time.perf_counter() - t0
     value = units / dt
     line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
@@ -903,7 +944,8 @@ def run_reference(args):
             "data": "synthetic",
             "config": {"workload": name, "sample_vectors_per_step": chunk},
             "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
-                             "sample": f"{chunk} vectors of the K cache per step, encode + decode"},
+                             "sample": f"{chunk} vectors of the K cache per step, encode + decode",
+                             "pinned": pin.pinned, **host_cpu()},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 

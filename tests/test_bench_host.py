@@ -38,3 +38,14 @@ def test_traffic_is_reported_only_for_the_source_it_was_taken_on():
             assert got is None
     assert bench.traffic_bytes("no_such_kernel", "kv") is None
     assert bench.traffic_bytes("tq3_decode", "no_such_workload") is None
+
+
+def test_oracle_timing_is_pinned_to_one_core_and_restored():
+    import bench
+    before = os.sched_getaffinity(0)
+    with bench.OneCore() as pin:
+        if pin.pinned:
+            assert len(os.sched_getaffinity(0)) == 1
+    assert os.sched_getaffinity(0) == before
+    info = bench.host_cpu()
+    assert info["nproc"] == len(before) and isinstance(info["cpu"], str)
