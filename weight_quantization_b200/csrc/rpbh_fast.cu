@@ -268,7 +268,8 @@ __global__ void __launch_bounds__(kMaxThreads)
 #pragma unroll
         for (int t = 0; t < G::S; ++t) {
             const float z = fb[bufpos<B>(blk, t, c)];
-            // correctly rounded z / den (Markstein: r = RN(1/den), q0 = RN(z r), e exact, RN(q0 + e r))
+            // z / den by Markstein's correction (r = RN(1/den), q0 = RN(z r), e = RN(z - q0 den),
+            // RN(q0 + e r)): correctly rounded for |z| >= 2^-100 and a normal quotient
             const float q0 = __fmul_rn(z, rden);
             const float u = __fmaf_rn(__fmaf_rn(-q0, den, z), rden, q0);
             raw[blk * G::H + c + (t << B)] = (uint8_t)bucketize<BITS, kSym>(u, E);
@@ -731,9 +732,9 @@ __global__ void __launch_bounds__(kSlotsT == 1 ? 128 : kMaxThreads, kSlotsT == 1
         const float den = __fadd_rn(rho, 1e-10f);
         const float rden = __frcp_rn(den);
         // codes, one byte each in element order, into the block's own part of the transpose buffer
-        // (its columns are in registers by now); u = z / den correctly rounded (Markstein:
-        // q0 = RN(z r), r = RN(1 / den), the remainder z - q0 den exact, u = RN(q0 + rem r)), two
-        // elements at a time
+        // (its columns are in registers by now); u = z / den by Markstein's correction
+        // (q0 = RN(z r), r = RN(1 / den), rem = RN(z - q0 den), u = RN(q0 + rem r)), correctly
+        // rounded for |z| >= 2^-100 and a normal quotient, two elements at a time
         const f32x2 RDEN = pk2(rden, rden), NDEN = pk2(-den, -den);
 #pragma unroll
         for (int k = 0; k < kSlots; ++k) {

@@ -400,8 +400,10 @@ __global__ void __maxnreg__(B == 4 ? 80 : 96)
             last_par = (uint32_t)(((it + 2) >> 1) & 1);
         }
         const float den = prm[set * 4 + 1], rden = prm[set * 4 + 2];
-        // u = z / den correctly rounded (q0 = RN(z r), the remainder z - q0 den exact, u = RN(q0 +
-        // rem r)), then the codes, one byte each in element order
+        // u = z / den by Markstein's correction (q0 = RN(z r), rem = RN(z - q0 den) by one fma,
+        // u = RN(q0 + rem r)): the correctly rounded quotient whenever |z| >= 2^-100 and z / den is
+        // a normal value, at most one unit in the last place off below that; then the codes, one
+        // byte each in element order
         const f32x2 RDEN = pk2(rden, rden), NDEN = pk2(-den, -den);
 #pragma unroll
         for (int k = 0; k < KS; ++k) {

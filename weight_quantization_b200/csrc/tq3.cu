@@ -13,10 +13,12 @@
 // operations are written explicitly only where they are exact), so packed bytes, norms and scales
 // are reproducible bit for bit:
 //   * the L2 norm sums exact fp64 squares and rounds the fp64 square root once to fp32;
-//   * x / n and xh / scale are correctly rounded quotients computed with Markstein's method: with
-//     r = RN(1/d), q0 = RN(x r), e = x - q0 d (exact by FMA), RN(q0 + e r) = RN(x / d)
-//     (P. Markstein, "Computation of elementary functions on the IBM RISC System/6000 processor",
-//     IBM J. Res. Dev. 34(1), 1990); it is checked bit for bit against IEEE division by the tests;
+//   * x / n and xh / scale are computed with Markstein's method: with r = RN(1/d),
+//     q0 = RN(x r), e = RN(x - q0 d) (one FMA), RN(q0 + e r) = RN(x / d) whenever |x| >= 2^-100
+//     and the quotient is a normal value (P. Markstein, "Computation of elementary functions on the
+//     IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990); below that the result can be
+//     one unit in the last place off (a unit of at least 2^-149), never of the other sign. The
+//     tests check the kernels bit for bit against IEEE division on vectors spanning 80 binades;
 //   * the butterflies and post-multipliers are single IEEE additions and multiplications (the
 //     last stage as one fused a * (+-1) + b, which rounds once like an addition);
 //   * the indices come from exact 0/1 saturated steps summed on the FMA pipe (add_index).
